@@ -1,0 +1,66 @@
+// Host-side declarations shared by the C-ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace msa {
+
+constexpr int kBlock = 128;      // KV block length of the method
+constexpr int kMaxTopk = 128;    // selection heap lives in shared memory
+constexpr int kMaxT = 1 << 20;   // per-tile block masks (nblk * 16 B) stay in shared memory
+
+// Device status word codes (first word of every workspace).  The high byte
+// says which kernel, the low bits which wait or check.
+enum : uint32_t {
+    kStOk = 0,
+    kStTimeoutBase = 0x100,      // + kernel id * 16 + wait id
+    kStIndexError = 0x8000,      // an idx entry outside [0, i/128]
+};
+enum KernelId : uint32_t { kKidProxy = 1, kKidFwd = 2, kKidBwd = 3, kKidDiag = 4 };
+
+struct Problem {
+    int B, T, Hq, Hkv, Hp, d, dp, topk, nblk, G;
+    float scale;
+    int64_t rows_q() const { return (int64_t)B * T * Hq; }
+};
+
+// Byte offsets of the workspace regions.
+struct WsLayout {
+    size_t status = 0;                           // 256 B: status word, index-error word
+    size_t cnt = 0, tot = 0, ptr = 0, tok = 0;   // block -> query inverse index
+    size_t qnorm = 0, kmax = 0, oacc = 0, lacc = 0, nflag = 0, flags = 0;   // forward
+    size_t dsum = 0, dqacc = 0;                  // backward
+    size_t total = 0;
+};
+WsLayout ws_layout(const Problem& p, int which);
+
+// Tensor map for a bf16 tensor [e3][e2][e1][e0] with a {box0, 1, box2, 1}
+// box and 128-byte swizzle.  Returns false if the driver refused it.
+bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t e0, uint64_t e1, uint64_t e2,
+                       uint64_t e3, uint32_t box0, uint32_t box2);
+
+// ---- launchers (return cudaGetLastError() of their launches) -------------
+cudaError_t launch_proxy_select(const Problem& p, const CUtensorMap& tm_qp, const CUtensorMap& tm_kp,
+                                int32_t* idx, int32_t* nsel, float* pooled, uint32_t* status,
+                                cudaStream_t st);
+
+cudaError_t launch_block_index(const Problem& p, const int32_t* idx, const int32_t* nsel, void* ws,
+                               const WsLayout& L, cudaStream_t st);
+
+cudaError_t launch_fwd(const Problem& p, const void* q, const void* k, const void* v,
+                       const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int32_t* idx,
+                       const int32_t* nsel, void* o, float* lse, void* ws, const WsLayout& L,
+                       cudaStream_t st);
+
+cudaError_t launch_bwd(const Problem& p, const void* q, const void* dout, const CUtensorMap& tm_k,
+                       const CUtensorMap& tm_v, const void* o, const float* lse, void* dq, void* dk,
+                       void* dv, void* ws, const WsLayout& L, cudaStream_t st);
+
+cudaError_t launch_diag_umma(int mode, int N, int K, const void* A, const void* B, float* D,
+                             uint32_t* status, cudaStream_t st);
+cudaError_t launch_diag_wait(uint64_t limit_ns, uint32_t* status, cudaStream_t st);
+
+}  // namespace msa

@@ -1,0 +1,464 @@
+// Main Branch backward: dQ, dK, dV of the block-sparse causal GQA attention
+// from dO, reusing the cached block selection and the forward's logsumexp.
+//
+// Method (ai-beat post on Flash-MSA training, paragraph 2: training through
+// the sparse pattern needs custom backward kernels; the selection itself is
+// piecewise constant, so no gradient reaches the proxy inputs).
+//
+// With P = exp(S - L), D_i = dO_i . O_i, dS = P (dO V^T - D) * scale:
+//   dV = P^T dO,  dK = dS^T Q,  dQ = dS K.
+//
+// KV-stationary: one CTA owns KV block n of one group, keeps K and V in
+// shared memory and dK, dV as fp32 accumulators in TMEM for the whole
+// bucket, so dK/dV need no atomics.  Chunks of 128 query rows (128/G tokens
+// x G heads) are gathered with cp.async (Q, dO, plus each row's L, D and
+// causal limit) into a 2-stage ring.  Per chunk, in the transposed
+// orientation so that one TMEM lane is one key:
+//   S^T = K Q^T, dP^T = V dO^T                 (tcgen05, A and B in smem)
+//   P^T, dS^T  -> TMEM (bf16) and dS^T -> smem  (softmax warps, lane = key)
+//   dV += P^T dO, dK += dS^T Q                  (tcgen05, A from TMEM)
+//   dQ_part = dS K                              (tcgen05, A = dS from smem)
+//   dQ_part -> fp32 reductions into a global accumulator (lane = query row).
+#include <math.h>
+
+#include "msa_device.cuh"
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 448;   // w0 TMA(K,V) | w1 MMA | w2-5 gather | w6-9 dS | w10-13 dQ, dK/dV out
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdParams {
+    int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
+    float c1;      // scale * log2(e)
+    float scale;
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* dout;
+    const float* lse;
+    const float* dsum;
+    const int32_t* ptr;
+    const int32_t* tok;
+    float* dqacc;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    uint32_t* status;
+};
+
+template <int D>
+struct BwdSmem {
+    static constexpr uint32_t kTile = 128u * D * 2u;
+    static constexpr uint32_t kK = 0, kV = kTile;
+    static constexpr uint32_t kStage0 = 2 * kTile;            // Q0, dO0, Q1, dO1
+    static constexpr uint32_t kDS = 6 * kTile;                 // dS tile (128 keys x 128 rows)
+    static constexpr uint32_t kMeta = kDS + 128 * 128 * 2;     // 2 x {L2[128], D[128], cmax[128]}
+    static constexpr uint32_t kMetaStage = 128 * 4 * 2 + 128;
+    static constexpr uint32_t kBars = kMeta + 2 * kMetaStage;
+    static constexpr uint32_t kNumBars = 12;
+    static constexpr uint32_t kTotal = kBars + kNumBars * 8 + 8;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                BwdParams p)
+{
+    using SM = BwdSmem<D>;
+    constexpr uint32_t kTile = SM::kTile;
+    constexpr int kSlabs = D / 64;
+    extern __shared__ __align__(1024) uint8_t smem[];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = p.B * p.Hkv;
+    const int n = (int)(blockIdx.x / BH), bg = (int)(blockIdx.x % BH);
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int G = 1 << p.lgG;
+    const int32_t* pp = p.ptr + (int64_t)bg * (p.nblk + 1);
+    const int beg = pp[n];
+    const int count = pp[n + 1] - beg;
+    const uint32_t code0 = kStTimeoutBase + kKidBwd * 16;
+
+    if (count <= 0) {
+        // no query reads this block: its dK, dV are zero
+        const int rows = min(128, p.T - n * 128);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        for (int x = threadIdx.x; x < rows * (D / 8); x += blockDim.x) {
+            const int j = n * 128 + x / (D / 8), e = (x % (D / 8)) * 8;
+            const int64_t off = (((int64_t)b * p.T + j) * p.Hkv + g) * D + e;
+            *reinterpret_cast<uint4*>(p.dk + off) = z;
+            *reinterpret_cast<uint4*>(p.dv + off) = z;
+        }
+        return;
+    }
+    if ((smem_u32(smem) & 1023u) != 0u) {   // the swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0) atomicCAS(p.status, 0u, code0 + 15);
+        return;
+    }
+    const int32_t* toks = p.tok + (int64_t)bg * p.T * p.topk + beg;
+    const int nchunks = (count + p.tpc - 1) / p.tpc;
+
+    uint8_t* k_tile = smem + SM::kK;
+    uint8_t* v_tile = smem + SM::kV;
+    uint8_t* ds_tile = smem + SM::kDS;
+    uint64_t* bars = (uint64_t*)(smem + SM::kBars);
+    uint64_t* kv_full = bars + 0;
+    uint64_t* st_full = bars + 1;    // [2]
+    uint64_t* st_empty = bars + 3;   // [2]
+    uint64_t* s_full = bars + 5;
+    uint64_t* p_full = bars + 6;
+    uint64_t* ds_empty = bars + 7;
+    uint64_t* dq_full = bars + 8;
+    uint64_t* dq_empty = bars + 9;
+    uint64_t* kv_done = bars + 10;
+    uint64_t* fin = bars + 11;
+    uint32_t* tmem_hold = (uint32_t*)(bars + SM::kNumBars);
+    volatile uint32_t* abort_flag = tmem_hold + 1;
+    const WaitCtx wc{p.status, abort_flag, MSA_WAIT_LIMIT_NS};
+
+    auto q_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kTile; };
+    auto do_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kTile + kTile; };
+    auto meta_l2 = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage); };
+    auto meta_d = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage + 512); };
+    auto meta_cm = [&](int s) { return (int8_t*)(smem + SM::kMeta + s * SM::kMetaStage + 1024); };
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < 2; ++s) { mbar_init(&st_full[s], 128); mbar_init(&st_empty[s], 1); }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(ds_empty, 1);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_empty, 128);
+        mbar_init(kv_done, 1);
+        mbar_init(fin, 1);
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 1) { tmem_alloc(tmem_hold, 512); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_hold;
+    // TMEM columns: S^T/P^T at 0, dP^T/dS^T/dQ at 128, dV at 256, dK at 256 + D.
+    const uint32_t tS = tmem, tdP = tmem + 128u, tdV = tmem + 256u, tdK = tmem + 256u + D;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            mbar_arrive_expect_tx(kv_full, 2 * kTile);
+            for (int s = 0; s < kSlabs; ++s) {
+                tma_load_4d(k_tile + s * 16384, &tm_k, kv_full, s * 64, g, n * 128, b);
+                tma_load_4d(v_tile + s * 16384, &tm_v, kv_full, s * 64, g, n * 128, b);
+            }
+            mbar_drain(kv_full, 0);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idSS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
+            constexpr uint32_t idKV = idesc_bf16(128, D, false, true);      // dV, dK (A in TMEM)
+            constexpr uint32_t idQ = idesc_bf16(128, D, true, true);        // dQ
+            const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile), dsa = smem_u32(ds_tile);
+            bool ok = mbar_wait(kv_full, 0, wc, code0 + 0);
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int s = c & 1;
+                const uint32_t su = (uint32_t)(c >> 1);
+                if (!mbar_wait(&st_full[s], su & 1u, wc, code0 + 1)) break;
+                if (c > 0 && !mbar_wait(dq_empty, (uint32_t)(c - 1) & 1u, wc, code0 + 2)) break;
+                tc_fence_after();
+                const uint32_t qa = smem_u32(q_stage(s)), oa = smem_u32(do_stage(s));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tS, desc_kmajor(ka, 128, kk * 16), desc_kmajor(qa, 128, kk * 16), idSS,
+                            kk > 0 ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tdP, desc_kmajor(va, 128, kk * 16), desc_kmajor(oa, 128, kk * 16), idSS,
+                            kk > 0 ? 1u : 0u);
+                umma_commit(s_full);
+                if (!mbar_wait(p_full, (uint32_t)c & 1u, wc, code0 + 3)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tdV, tS + kk * 8, desc_mnmajor(oa, 128, kk * 16), idKV,
+                            (c > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tdK, tdP + kk * 8, desc_mnmajor(qa, 128, kk * 16), idKV,
+                            (c > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ss(tdP, desc_mnmajor(dsa, 128, kk * 16), desc_mnmajor(ka, 128, kk * 16), idQ,
+                            kk > 0 ? 1u : 0u);
+                umma_commit(&st_empty[s]);
+                umma_commit(ds_empty);
+                umma_commit(dq_full);
+            }
+            umma_commit(kv_done);
+            umma_commit(fin);
+            mbar_drain(fin, 0);
+        }
+    } else if (warp < 6) {
+        // ---------------- gather Q, dO and per-row metadata ----------------
+        const int tid = threadIdx.x - 64;
+        constexpr int kPieces = 128 * D / 8;
+        constexpr int kRowPieces = D / 8;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const uint32_t su = (uint32_t)(c >> 1);
+            if (su > 0 && !mbar_wait(&st_empty[s], (su - 1) & 1u, wc, code0 + 4)) break;
+            const uint32_t qs = smem_u32(q_stage(s)), os = smem_u32(do_stage(s));
+#pragma unroll 4
+            for (int it = 0; it < kPieces / 128; ++it) {
+                const int piece = it * 128 + tid;
+                const int row = piece / kRowPieces, ch = piece % kRowPieces;
+                const int t = row >> p.lgG, hh = row & (G - 1);
+                const int jj = c * p.tpc + t;
+                const bool valid = jj < count;
+                const int i = valid ? toks[jj] : 0;
+                const int64_t off = (((int64_t)b * p.T + i) * p.Hq + g * G + hh) * D + ch * 8;
+                const uint32_t dst = sw128_offset(row, ch & 7, ch >> 3, 128);
+                cp_async_16(qs + dst, p.q + off, valid ? 16u : 0u);
+                cp_async_16(os + dst, p.dout + off, valid ? 16u : 0u);
+            }
+            {
+                const int row = tid;
+                const int t = row >> p.lgG, hh = row & (G - 1), h = g * G + hh;
+                const int jj = c * p.tpc + t;
+                const bool valid = jj < count;
+                const int i = valid ? toks[jj] : 0;
+                const int64_t lrow = ((int64_t)b * p.Hq + h) * p.T + i;
+                meta_l2(s)[row] = valid ? p.lse[lrow] * kLog2e : 0.f;
+                meta_d(s)[row] = valid ? p.dsum[lrow] : 0.f;
+                meta_cm(s)[row] = (int8_t)(valid ? (((i >> 7) == n) ? (i & 127) : 127) : -1);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&st_full[s]);
+        }
+        cp_async_wait<0>();
+    } else if (warp < 10) {
+        // ---------------- P^T, dS^T (one TMEM lane = one key) ----------------
+        const int jl = ((warp & 3) << 5) | lane;   // key within the block
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        const uint32_t aS = tmem_addr(tS, lane_base, 0), aP = tmem_addr(tdP, lane_base, 0);
+        const uint32_t dsa = smem_u32(ds_tile);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            bool ok = mbar_wait(s_full, (uint32_t)c & 1u, wc, code0 + 5);
+            if (ok && c > 0) ok = mbar_wait(ds_empty, (uint32_t)(c - 1) & 1u, wc, code0 + 6);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const float* L2 = meta_l2(s);
+            const float* Dv = meta_d(s);
+            const int8_t* cm = meta_cm(s);
+#pragma unroll
+            for (int piece = 0; piece < 4; ++piece) {
+                uint32_t sv[32], dv[32], pk[16], dk[16];
+                tmem_ld32(aS + piece * 32, sv);
+                tmem_ld32(aP + piece * 32, dv);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int r0 = piece * 32 + 2 * e, r1 = r0 + 1;
+                    const float p0 = jl <= (int)cm[r0]
+                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e]), p.c1, -L2[r0]))
+                                         : 0.f;
+                    const float p1 = jl <= (int)cm[r1]
+                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), p.c1, -L2[r1]))
+                                         : 0.f;
+                    const float d0 = p0 * (__uint_as_float(dv[2 * e]) - Dv[r0]) * p.scale;
+                    const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - Dv[r1]) * p.scale;
+                    pk[e] = pack_bf16x2(p0, p1);
+                    dk[e] = pack_bf16x2(d0, d1);
+                }
+                tmem_st16(aS + piece * 16, pk);   // P^T over S^T columns already read
+                tmem_st16(aP + piece * 16, dk);   // dS^T over dP^T columns already read
+                // dS^T row jl (rows piece*32 .. +31) into the MN-major dS tile
+                const uint32_t slab = (uint32_t)piece >> 1, cb = ((uint32_t)piece & 1u) * 4u;
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const uint32_t addr = dsa + sw128_offset((uint32_t)jl, cb + qd, slab, 128);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * qd]),
+                                 "r"(dk[4 * qd + 1]), "r"(dk[4 * qd + 2]), "r"(dk[4 * qd + 3])
+                                 : "memory");
+                }
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+    } else {
+        // ---------------- dQ partials out; dK, dV at the end ----------------
+        const int r = ((warp & 3) << 5) | lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
+        bool ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            ok = mbar_wait(dq_full, (uint32_t)c & 1u, wc, code0 + 7);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            const int jj = c * p.tpc + t;
+            const bool valid = jj < count;
+            const int i = valid ? toks[jj] : 0;
+            float* dst = p.dqacc + (((int64_t)b * p.T + i) * p.Hq + h) * D;
+            const uint32_t ta = tmem_addr(tdP, lane_base, 0);
+#pragma unroll
+            for (int piece = 0; piece < D / 32; ++piece) {
+                uint32_t v[32];
+                tmem_ld32(ta + piece * 32, v);
+                tmem_ld_wait();
+                if (valid) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        red_add_v4(dst + piece * 32 + 4 * e, __uint_as_float(v[4 * e]),
+                                   __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
+                                   __uint_as_float(v[4 * e + 3]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(dq_empty);
+        }
+        if (ok) ok = mbar_wait(kv_done, 0, wc, code0 + 8);
+        if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            const int j = n * 128 + r;   // this lane's key
+            const int64_t off = (((int64_t)b * p.T + j) * p.Hkv + g) * D;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t ta = tmem_addr(which == 0 ? tdV : tdK, lane_base, 0);
+                __nv_bfloat16* out = (which == 0 ? p.dv : p.dk) + off;
+#pragma unroll
+                for (int piece = 0; piece < D / 32; ++piece) {
+                    uint32_t v[32];
+                    tmem_ld32(ta + piece * 32, v);
+                    tmem_ld_wait();
+                    if (j < p.T) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            uint4 u;
+                            u.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]), __uint_as_float(v[8 * e + 1]));
+                            u.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3]));
+                            u.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5]));
+                            u.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7]));
+                            *reinterpret_cast<uint4*>(out + piece * 32 + 8 * e) = u;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// D_i = dO_i . O_i per query row (bf16 inputs, fp32 sum); D/8 lanes per row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dsum_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout, int B, int T,
+                                                       int Hq, float* __restrict__ dsum)
+{
+    constexpr int LPR = D / 8;
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt / LPR;
+    const int sub = (int)(gt % LPR);
+    const bool ok = row < (int64_t)B * T * Hq;
+    float s = 0.f;
+    if (ok) {
+        const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + sub * 8);
+        const uint4 c = *reinterpret_cast<const uint4*>(dout + row * D + sub * 8);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 x = __bfloat1622float2(a2[e]), y = __bfloat1622float2(c2[e]);
+            s = fmaf(x.x, y.x, s);
+            s = fmaf(x.y, y.y, s);
+        }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (ok && sub == 0) {
+        const int h = (int)(row % Hq);
+        const int64_t bi = row / Hq;
+        const int i = (int)(bi % T), b = (int)(bi / T);
+        dsum[((int64_t)b * Hq + h) * T + i] = s;
+    }
+}
+
+// fp32 dQ accumulator -> bf16, 8 elements per thread.
+__global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __restrict__ acc,
+                                                             __nv_bfloat16* __restrict__ dq, int64_t n8)
+{
+    const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= n8) return;
+    const float4 a = *reinterpret_cast<const float4*>(acc + x * 8);
+    const float4 c = *reinterpret_cast<const float4*>(acc + x * 8 + 4);
+    uint4 u;
+    u.x = pack_bf16x2(a.x, a.y);
+    u.y = pack_bf16x2(a.z, a.w);
+    u.z = pack_bf16x2(c.x, c.y);
+    u.w = pack_bf16x2(c.z, c.w);
+    *reinterpret_cast<uint4*>(dq + x * 8) = u;
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, const CUtensorMap& tm_k,
+                         const CUtensorMap& tm_v, const void* o, const float* lse, void* dq, void* dk,
+                         void* dv, void* ws, const WsLayout& L, cudaStream_t st)
+{
+    uint8_t* w = (uint8_t*)ws;
+    float* dsum = (float*)(w + L.dsum);
+    float* dqacc = (float*)(w + L.dqacc);
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(dqacc, 0, sizeof(float) * (size_t)pr.rows_q() * D, st)) != cudaSuccess)
+        return e;
+    const int64_t th = pr.rows_q() * (D / 8);
+    bwd_dsum_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, dsum);
+
+    BwdParams p;
+    p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
+    p.lgG = 31 - __builtin_clz((unsigned)pr.G);
+    p.tpc = 128 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;
+    p.c1 = pr.scale * kLog2e;
+    p.scale = pr.scale;
+    p.q = (const __nv_bfloat16*)q;
+    p.dout = (const __nv_bfloat16*)dout;
+    p.lse = lse;
+    p.dsum = dsum;
+    p.ptr = (const int32_t*)(w + L.ptr);
+    p.tok = (const int32_t*)(w + L.tok);
+    p.dqacc = dqacc;
+    p.dk = (__nv_bfloat16*)dk;
+    p.dv = (__nv_bfloat16*)dv;
+    p.status = (uint32_t*)(w + L.status);
+    const size_t smem = BwdSmem<D>::kTotal;
+    if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+        return e;
+    bwd_main_kernel<D><<<(unsigned)(pr.nblk * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+    const int64_t n8 = pr.rows_q() * D / 8;
+    bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dqacc, (__nv_bfloat16*)dq, n8);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const Problem& pr, const void* q, const void* dout, const CUtensorMap& tm_k,
+                       const CUtensorMap& tm_v, const void* o, const float* lse, void* dq, void* dk,
+                       void* dv, void* ws, const WsLayout& L, cudaStream_t st)
+{
+    if (pr.d == 64) return launch_bwd_d<64>(pr, q, dout, tm_k, tm_v, o, lse, dq, dk, dv, ws, L, st);
+    return launch_bwd_d<128>(pr, q, dout, tm_k, tm_v, o, lse, dq, dk, dv, ws, L, st);
+}
+
+}  // namespace msa

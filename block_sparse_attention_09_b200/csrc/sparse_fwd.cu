@@ -1,0 +1,498 @@
+// Main Branch forward: exact causal softmax attention (GQA) over the cached
+// block selection, producing O and the logsumexp L.
+//
+// Method (ai-beat post on Flash-MSA training, paragraph 1: the Main Branch
+// runs exact softmax over only the selected blocks; "Flash-MSA: Open-Source
+// Sparse Attention Kernels Debut", section "How MSA works": GQA main
+// attention, block ids cached by the Index Branch).
+//
+// KV-stationary design.  One CTA owns one KV block n of one group: its K and
+// V tiles (128 keys) are loaded once by TMA; the queries that selected the
+// block are gathered from the inverse index in chunks of 128 rows (128/G
+// tokens x the G query heads of the group) with cp.async into a 3-stage ring.
+// Per chunk:  S = Q K^T (tcgen05, TMEM) -> P = exp(S*scale - bound) written
+// back to TMEM as bf16 -> O_part = P V (tcgen05 with A from TMEM) -> fp32
+// reductions of O_part and of the row sums into global accumulators.
+//
+// Softmax normalisation across the CTAs that share a query row uses a fixed
+// per-row shift instead of a running maximum: the Cauchy-Schwarz bound
+// |scale| * |q_i| * max_j |k_j| is never below any score, so exp(S - bound)
+// cannot overflow and every CTA's partial sums are directly additive.  The
+// finalize pass divides by the row sum and sets L = bound + log(sum).  Rows
+// whose sum underflows (bound far above the true maximum) are listed and
+// recomputed exactly by a fallback kernel with a two-pass softmax.
+#include <math.h>
+
+#include "msa_device.cuh"
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kThreads = 448;   // w0 TMA(K,V) | w1 MMA | w2-5 gather | w6-9 softmax | w10-13 O out
+constexpr int kQStages = 3;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kUnderflow = 5.421010862427522e-20f;   // 2^-64: row sums below are redone exactly
+
+struct FwdParams {
+    int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
+    float c1;        // scale * log2(e)
+    float bound;     // |scale| * log2(e)
+    const __nv_bfloat16* q;
+    const int32_t* ptr;
+    const int32_t* tok;
+    const float* qn;
+    const float* kmax;
+    float* oacc;
+    float* lacc;
+    uint32_t* status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                FwdParams p)
+{
+    constexpr uint32_t kTile = 128u * D * 2u;   // 128 rows x D bf16
+    constexpr int kSlabs = D / 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = p.B * p.Hkv;
+    const int n = (int)(blockIdx.x / BH), bg = (int)(blockIdx.x % BH);   // low blocks (most selected) first
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int G = 1 << p.lgG;
+    const int32_t* pp = p.ptr + (int64_t)bg * (p.nblk + 1);
+    const int beg = pp[n];
+    const int count = pp[n + 1] - beg;
+    if (count <= 0) return;
+    const int32_t* toks = p.tok + (int64_t)bg * p.T * p.topk + beg;
+    const int nchunks = (count + p.tpc - 1) / p.tpc;
+
+    uint8_t* k_tile = smem;
+    uint8_t* v_tile = smem + kTile;
+    uint8_t* q_st = smem + 2 * kTile;
+    uint64_t* bars = (uint64_t*)(q_st + kQStages * kTile);
+    uint64_t* kv_full = bars;
+    uint64_t* q_full = bars + 1;
+    uint64_t* q_empty = q_full + kQStages;
+    uint64_t* s_full = q_empty + kQStages;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* o_full = p_full + 2;
+    uint64_t* o_empty = o_full + 2;
+    uint64_t* fin = o_empty + 2;
+    uint32_t* tmem_hold = (uint32_t*)(fin + 1);
+    volatile uint32_t* abort_flag = tmem_hold + 1;
+    const WaitCtx wc{p.status, abort_flag, MSA_WAIT_LIMIT_NS};
+    const uint32_t code0 = kStTimeoutBase + kKidFwd * 16;
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < kQStages; ++s) { mbar_init(&q_full[s], 128); mbar_init(&q_empty[s], 1); }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], 128);
+            mbar_init(&o_full[s], 1);
+            mbar_init(&o_empty[s], 128);
+        }
+        mbar_init(fin, 1);
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 1) { tmem_alloc(tmem_hold, 512); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_hold;
+    // TMEM columns: S/P buffers at 0 and 128, O buffers at 256 and 256 + D.
+
+    if (warp == 0) {
+        // ---------------- K/V tiles (once) ----------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            mbar_arrive_expect_tx(kv_full, 2 * kTile);
+            for (int s = 0; s < kSlabs; ++s) {
+                tma_load_4d(k_tile + s * 16384, &tm_k, kv_full, s * 64, g, n * 128, b);
+                tma_load_4d(v_tile + s * 16384, &tm_v, kv_full, s * 64, g, n * 128, b);
+            }
+            mbar_drain(kv_full, 0);   // the tiles must have landed before this warp leaves
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idPV = idesc_bf16(128, D, false, true);
+            const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile), qa = smem_u32(q_st);
+            auto issue_s = [&](int c) -> bool {
+                const int s = c % kQStages;
+                const uint32_t use = (uint32_t)(c / kQStages);
+                if (!mbar_wait(&q_full[s], use & 1u, wc, code0 + 1)) return false;
+                tc_fence_after();
+                const uint32_t qs = qa + s * kTile;
+                const uint32_t dS = tmem + (uint32_t)(c & 1) * 128u;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(dS, desc_kmajor(qs, 128, kk * 16), desc_kmajor(ka, 128, kk * 16), idS,
+                            kk > 0 ? 1u : 0u);
+                umma_commit(&q_empty[s]);
+                umma_commit(&s_full[c & 1]);
+                return true;
+            };
+            bool ok = mbar_wait(kv_full, 0, wc, code0 + 0);
+            if (ok && nchunks > 0) ok = issue_s(0);
+            if (ok && nchunks > 1) ok = issue_s(1);
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int buf = c & 1;
+                const uint32_t use = (uint32_t)(c >> 1);
+                if (!mbar_wait(&p_full[buf], use & 1u, wc, code0 + 2)) break;
+                if (use > 0 && !mbar_wait(&o_empty[buf], (use - 1) & 1u, wc, code0 + 3)) break;
+                tc_fence_after();
+                const uint32_t pa = tmem + (uint32_t)buf * 128u;
+                const uint32_t oa = tmem + 256u + (uint32_t)buf * D;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(oa, pa + kk * 8, desc_mnmajor(va, 128, kk * 16), idPV, kk > 0 ? 1u : 0u);
+                umma_commit(&o_full[buf]);
+                if (c + 2 < nchunks) ok = issue_s(c + 2);
+            }
+            umma_commit(fin);
+            mbar_drain(fin, 0);
+        }
+    } else if (warp < 6) {
+        // ---------------- query gather (cp.async, 128 threads) ----------------
+        const int tid = threadIdx.x - 64;
+        constexpr int kPieces = 128 * D / 8;           // 16-byte pieces per chunk
+        constexpr int kRowPieces = D / 8;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kQStages;
+            const uint32_t use = (uint32_t)(c / kQStages);
+            if (use > 0 && !mbar_wait(&q_empty[s], (use - 1) & 1u, wc, code0 + 4)) break;
+            const uint32_t qs = smem_u32(q_st + s * kTile);
+#pragma unroll 4
+            for (int it = 0; it < kPieces / 128; ++it) {
+                const int piece = it * 128 + tid;
+                const int row = piece / kRowPieces, ch = piece % kRowPieces;
+                const int t = row >> p.lgG, hh = row & (G - 1);
+                const int jj = c * p.tpc + t;
+                const bool valid = jj < count;
+                const int i = valid ? toks[jj] : 0;
+                const __nv_bfloat16* src =
+                    p.q + (((int64_t)b * p.T + i) * p.Hq + g * G + hh) * D + ch * 8;
+                cp_async_16(qs + sw128_offset(row, ch & 7, ch >> 3, 128), src, valid ? 16u : 0u);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&q_full[s]);
+        }
+        cp_async_wait<0>();
+    } else if (warp < 10) {
+        // ---------------- softmax: P = exp2(S*c1 - bound) ----------------
+        const int r = ((warp & 3) << 5) | lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
+        const float kmx = p.kmax[bg];
+        for (int c = 0; c < nchunks; ++c) {
+            const int buf = c & 1;
+            const uint32_t use = (uint32_t)(c >> 1);
+            const bool ok = mbar_wait(&s_full[buf], use & 1u, wc, code0 + 5);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int jj = c * p.tpc + t;
+            const bool valid = jj < count;
+            const int i = valid ? toks[jj] : 0;
+            const int cmax = valid ? (((i >> 7) == n) ? (i & 127) : 127) : -1;
+            const float mh = valid ? p.bound * p.qn[((int64_t)b * p.Hq + h) * p.T + i] * kmx : 0.f;
+            const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 128u);
+            float l = 0.f;
+#pragma unroll
+            for (int piece = 0; piece < 4; ++piece) {
+                uint32_t v[32], pk[16];
+                tmem_ld32(ta + piece * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int c0 = piece * 32 + 2 * e;
+                    const float p0 = c0 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e]), p.c1, -mh)) : 0.f;
+                    const float p1 = c0 + 1 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mh)) : 0.f;
+                    pk[e] = pack_bf16x2(p0, p1);
+                    // normalise by the weights the PV product actually uses (bf16), so
+                    // that O is an exact convex combination of the selected values
+                    l += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+                }
+                tmem_st16(ta + piece * 16, pk);   // P overwrites S columns already read
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_full[buf]);
+            if (valid) atomicAdd(&p.lacc[((int64_t)b * p.Hq + h) * p.T + i], l);
+        }
+    } else {
+        // ---------------- O partials -> fp32 global accumulators ----------------
+        const int r = ((warp & 3) << 5) | lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
+        for (int c = 0; c < nchunks; ++c) {
+            const int buf = c & 1;
+            const uint32_t use = (uint32_t)(c >> 1);
+            const bool ok = mbar_wait(&o_full[buf], use & 1u, wc, code0 + 6);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int jj = c * p.tpc + t;
+            const bool valid = jj < count;
+            const int i = valid ? toks[jj] : 0;
+            float* dst = p.oacc + (((int64_t)b * p.T + i) * p.Hq + h) * D;
+            const uint32_t ta = tmem_addr(tmem, lane_base, 256u + (uint32_t)buf * D);
+#pragma unroll
+            for (int piece = 0; piece < D / 32; ++piece) {
+                uint32_t v[32];
+                tmem_ld32(ta + piece * 32, v);
+                tmem_ld_wait();
+                if (valid) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        red_add_v4(dst + piece * 32 + 4 * e, __uint_as_float(v[4 * e]),
+                                   __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
+                                   __uint_as_float(v[4 * e + 3]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&o_empty[buf]);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// |q| per query row and max |k| per (b, group).  D/8 lanes per row.
+template <int D>
+__global__ void __launch_bounds__(256) fwd_norms_kernel(const __nv_bfloat16* __restrict__ q,
+                                                        const __nv_bfloat16* __restrict__ k, int B, int T,
+                                                        int Hq, int Hkv, float* __restrict__ qn,
+                                                        uint32_t* __restrict__ kmax_bits)
+{
+    constexpr int LPR = D / 8;
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt / LPR;
+    const int sub = (int)(gt % LPR);
+    const int64_t nq = (int64_t)B * T * Hq, nk = (int64_t)B * T * Hkv;
+    const bool isq = row < nq, isk = !isq && row < nq + nk;
+    float ss = 0.f;
+    if (isq || isk) {
+        const __nv_bfloat16* src = isq ? q + row * D : k + (row - nq) * D;
+        const uint4 u = *reinterpret_cast<const uint4*>(src + sub * 8);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            ss = fmaf(f.x, f.x, ss);
+            ss = fmaf(f.y, f.y, ss);
+        }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (sub == 0) {
+        if (isq) {
+            const int h = (int)(row % Hq);
+            const int64_t bi = row / Hq;
+            const int i = (int)(bi % T), b = (int)(bi / T);
+            qn[((int64_t)b * Hq + h) * T + i] = sqrtf(ss);
+        } else if (isk) {
+            const int64_t kr = row - nq;
+            const int gg = (int)(kr % Hkv);
+            const int b = (int)(kr / Hkv / T);
+            atomicMax(&kmax_bits[b * Hkv + gg], __float_as_uint(sqrtf(ss)));
+        }
+    }
+}
+
+// O = O_acc / l (bf16), L = bound + log(l); rows whose l underflowed are listed.
+template <int D>
+__global__ void __launch_bounds__(256) fwd_finalize_kernel(const float* __restrict__ oacc,
+                                                           const float* __restrict__ lacc,
+                                                           const float* __restrict__ qn,
+                                                           const float* __restrict__ kmax, int B, int T,
+                                                           int Hq, int Hkv, float abs_scale,
+                                                           __nv_bfloat16* __restrict__ o,
+                                                           float* __restrict__ lse, int* nflag,
+                                                           int* flags)
+{
+    constexpr int LPR = D / 8;
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = gt / LPR;   // (b*T + i)*Hq + h
+    const int sub = (int)(gt % LPR);
+    if (row >= (int64_t)B * T * Hq) return;
+    const int h = (int)(row % Hq);
+    const int64_t bi = row / Hq;
+    const int i = (int)(bi % T), b = (int)(bi / T);
+    const int G = Hq / Hkv;
+    const int64_t lrow = ((int64_t)b * Hq + h) * T + i;
+    const float l = lacc[lrow];
+    const float inv = 1.f / l;
+    const float4 a = *reinterpret_cast<const float4*>(oacc + row * D + sub * 8);
+    const float4 c = *reinterpret_cast<const float4*>(oacc + row * D + sub * 8 + 4);
+    uint4 out;
+    out.x = pack_bf16x2(a.x * inv, a.y * inv);
+    out.y = pack_bf16x2(a.z * inv, a.w * inv);
+    out.z = pack_bf16x2(c.x * inv, c.y * inv);
+    out.w = pack_bf16x2(c.z * inv, c.w * inv);
+    *reinterpret_cast<uint4*>(o + row * D + sub * 8) = out;
+    if (sub == 0) {
+        const float mh = abs_scale * qn[lrow] * kmax[b * Hkv + h / G];
+        lse[lrow] = mh + logf(l);
+        if (!(l >= kUnderflow)) flags[atomicAdd(nflag, 1)] = (int)row;
+    }
+}
+
+// Exact two-pass softmax for the listed rows (rare: bound far above the true
+// maximum).  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(128) fwd_fallback_kernel(const __nv_bfloat16* __restrict__ q,
+                                                           const __nv_bfloat16* __restrict__ k,
+                                                           const __nv_bfloat16* __restrict__ v,
+                                                           const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ nsel, int B, int T,
+                                                           int Hq, int Hkv, int topk, float scale,
+                                                           const int* nflag, const int* flags,
+                                                           __nv_bfloat16* __restrict__ o,
+                                                           float* __restrict__ lse)
+{
+    __shared__ float qs[4][D];
+    __shared__ float ps[4][32];
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = Hq / Hkv;
+    const int nf = *nflag;
+    for (int f = blockIdx.x * 4 + w; f < nf; f += gridDim.x * 4) {
+        const int64_t row = flags[f];
+        const int h = (int)(row % Hq);
+        const int64_t bi = row / Hq;
+        const int i = (int)(bi % T), b = (int)(bi / T);
+        const int g = h / G, bg = b * Hkv + g;
+        for (int e = lane; e < D; e += 32) qs[w][e] = __bfloat162float(q[row * D + e]);
+        __syncwarp();
+        const int64_t srow = (int64_t)bg * T + i;
+        int ns = nsel[srow];
+        ns = ns < 0 ? 0 : (ns > topk ? topk : ns);
+        const int32_t* sel = idx + srow * topk;
+        auto score = [&](int j) {
+            const __nv_bfloat16* kr = k + (((int64_t)b * T + j) * Hkv + g) * D;
+            float acc = 0.f;
+            for (int e = 0; e < D; ++e) acc = fmaf(qs[w][e], __bfloat162float(kr[e]), acc);
+            return acc * scale;
+        };
+        float m = -INFINITY;
+        int prev = -1;
+        for (int s = 0; s < ns; ++s) {
+            const int nb = sel[s];
+            if (nb < 0 || nb > (i >> 7) || nb <= prev) continue;
+            prev = nb;
+            const int jend = min(nb * 128 + 128, i + 1);
+            for (int j = nb * 128 + lane; j < jend; j += 32) m = fmaxf(m, score(j));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float l = 0.f, acc[D / 32];
+#pragma unroll
+        for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+        prev = -1;
+        for (int s = 0; s < ns; ++s) {
+            const int nb = sel[s];
+            if (nb < 0 || nb > (i >> 7) || nb <= prev) continue;
+            prev = nb;
+            const int jend = min(nb * 128 + 128, i + 1);
+            for (int jb = nb * 128; jb < jend; jb += 32) {
+                const int j = jb + lane;
+                const float pe = j < jend ? expf(score(j) - m) : 0.f;
+                l += pe;
+                ps[w][lane] = pe;
+                __syncwarp();
+                const int cnt = min(32, jend - jb);
+                for (int kk = 0; kk < cnt; ++kk) {
+                    const __nv_bfloat16* vr = v + (((int64_t)b * T + jb + kk) * Hkv + g) * D;
+#pragma unroll
+                    for (int e = 0; e < D / 32; ++e)
+                        acc[e] = fmaf(ps[w][kk], __bfloat162float(vr[lane + 32 * e]), acc[e]);
+                }
+                __syncwarp();
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+#pragma unroll
+        for (int e = 0; e < D / 32; ++e) o[row * D + lane + 32 * e] = __float2bfloat16(acc[e] / l);
+        if (lane == 0) lse[((int64_t)b * Hq + h) * T + i] = m + logf(l);
+        __syncwarp();
+    }
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const void* v,
+                         const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int32_t* idx,
+                         const int32_t* nsel, void* o, float* lse, void* ws, const WsLayout& L,
+                         cudaStream_t st)
+{
+    uint8_t* w = (uint8_t*)ws;
+    float* qn = (float*)(w + L.qnorm);
+    float* kmax = (float*)(w + L.kmax);
+    float* oacc = (float*)(w + L.oacc);
+    float* lacc = (float*)(w + L.lacc);
+    int* nflag = (int*)(w + L.nflag);
+    int* flags = (int*)(w + L.flags);
+    const __nv_bfloat16* qb = (const __nv_bfloat16*)q;
+    const __nv_bfloat16* kb = (const __nv_bfloat16*)k;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(kmax, 0, sizeof(float) * pr.B * pr.Hkv, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(oacc, 0, sizeof(float) * (size_t)pr.rows_q() * D, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(lacc, 0, sizeof(float) * (size_t)pr.rows_q(), st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(nflag, 0, sizeof(int), st)) != cudaSuccess) return e;
+
+    const int64_t nrows = (int64_t)pr.B * pr.T * (pr.Hq + pr.Hkv);
+    const int64_t th = nrows * (D / 8);
+    fwd_norms_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(qb, kb, pr.B, pr.T, pr.Hq, pr.Hkv, qn,
+                                                                     (uint32_t*)kmax);
+
+    FwdParams p;
+    p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
+    p.lgG = 31 - __builtin_clz((unsigned)pr.G);
+    p.tpc = 128 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;
+    p.c1 = pr.scale * kLog2e;
+    p.bound = fabsf(pr.scale) * kLog2e;
+    p.q = qb;
+    p.ptr = (const int32_t*)(w + L.ptr);
+    p.tok = (const int32_t*)(w + L.tok);
+    p.qn = qn; p.kmax = kmax; p.oacc = oacc; p.lacc = lacc;
+    p.status = (uint32_t*)(w + L.status);
+    const size_t smem = 1024 + (size_t)(2 + kQStages) * 128 * D * 2 + 32 * 8;
+    if ((e = cudaFuncSetAttribute(fwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+        return e;
+    fwd_main_kernel<D><<<(unsigned)(pr.nblk * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+
+    const int64_t fth = (int64_t)pr.rows_q() * (D / 8);
+    fwd_finalize_kernel<D><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(
+        oacc, lacc, qn, kmax, pr.B, pr.T, pr.Hq, pr.Hkv, fabsf(pr.scale), (__nv_bfloat16*)o, lse, nflag,
+        flags);
+    fwd_fallback_kernel<D><<<148, 128, 0, st>>>(qb, kb, (const __nv_bfloat16*)v, idx, nsel, pr.B,
+                                                pr.T, pr.Hq, pr.Hkv, pr.topk, pr.scale, nflag, flags,
+                                                (__nv_bfloat16*)o, lse);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const Problem& pr, const void* q, const void* k, const void* v,
+                       const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int32_t* idx,
+                       const int32_t* nsel, void* o, float* lse, void* ws, const WsLayout& L,
+                       cudaStream_t st)
+{
+    if (pr.d == 64) return launch_fwd_d<64>(pr, q, k, v, tm_k, tm_v, idx, nsel, o, lse, ws, L, st);
+    return launch_fwd_d<128>(pr, q, k, v, tm_k, tm_v, idx, nsel, o, lse, ws, L, st);
+}
+
+}  // namespace msa

@@ -1,0 +1,206 @@
+"""Thin Python binding of libmsa.so (the C ABI in include/msa.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  There is no
+CPU or PyTorch fallback: if libmsa.so is missing the import fails.
+
+    from block_sparse_attention_09_b200 import msa
+    idx, nsel = msa.proxy_select(qp, kp, topk)              # Index Branch (cached)
+    o, lse = msa.fwd(q, k, v, idx, nsel)                     # Main Branch forward
+    dq, dk, dv = msa.bwd(q, k, v, o, dout, lse, idx, nsel)   # Main Branch backward
+    o = msa.MSAAttention.apply(q, k, v, qp, kp, topk)        # autograd wrapper
+
+Layouts: q, o, dout [B,T,Hq,d]; k, v [B,T,Hkv,d]; qp, kp [B,T,Hkv,dp], all
+bf16 and contiguous; idx [B,Hkv,T,topk] int32; nsel [B,Hkv,T] int32;
+lse [B,Hq,T] fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+MSA_SELECT, MSA_FWD, MSA_BWD = 0, 1, 2
+_ERR = {0: "ok", -1: "invalid dimensions", -2: "null pointer", -3: "misaligned pointer",
+        -4: "workspace too small", -5: "CUDA launch failed", -6: "device wait timed out",
+        -7: "device is not sm_100", -8: "tensor map encoding failed",
+        -9: "block index out of range"}
+
+
+class MsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {_ERR.get(code, 'unknown')} ({code})")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("Hp", ctypes.c_int), ("d", ctypes.c_int), ("dp", ctypes.c_int), ("block", ctypes.c_int),
+                ("topk", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmsa.so not built ({LIB_PATH}); run `python -m block_sparse_attention_09_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, SZ, I, U64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint64
+    D = ctypes.POINTER(Dims)
+    lib.msa_workspace_size.argtypes = [D, I]
+    lib.msa_workspace_size.restype = SZ
+    lib.msa_proxy_select.argtypes = [D, P, P, P, P, P, P, SZ, P]
+    lib.msa_fwd.argtypes = [D, P, P, P, P, P, P, P, P, SZ, P]
+    lib.msa_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    lib.msa_check_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.msa_strerror.argtypes = [I]
+    lib.msa_strerror.restype = ctypes.c_char_p
+    lib.msa_diag_umma.argtypes = [I, I, I, P, P, P, P, P]
+    lib.msa_diag_wait_timeout.argtypes = [U64, P, P]
+    for f in ("msa_proxy_select", "msa_fwd", "msa_bwd", "msa_check_status", "msa_diag_umma",
+              "msa_diag_wait_timeout"):
+        getattr(lib, f).restype = I
+    return lib
+
+
+LIB = _load()
+
+
+def make_dims(B, T, Hq, Hkv, d, dp, topk, scale=0.0) -> Dims:
+    return Dims(int(B), int(T), int(Hq), int(Hkv), int(Hkv), int(d), int(dp), 128, int(topk), float(scale))
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc, where):
+    if rc != 0:
+        raise MsaError(rc, where)
+
+
+def workspace_size(dims: Dims, which: int) -> int:
+    return int(LIB.msa_workspace_size(ctypes.byref(dims), which))
+
+
+def workspace(dims: Dims, which: int, device) -> torch.Tensor:
+    return torch.empty(max(workspace_size(dims, which), 256), dtype=torch.uint8, device=device)
+
+
+def check_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise and read the status word a call left in ``ws``."""
+    code = ctypes.c_uint32(0)
+    rc = LIB.msa_check_status(_p(ws), _stream(stream), ctypes.byref(code))
+    return rc
+
+
+def _bf16(*ts):
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("expected contiguous CUDA bf16 tensors")
+
+
+def dims_of(q, k, qp, topk, scale=0.0) -> Dims:
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    dp = qp.shape[3] if qp is not None else 64
+    return make_dims(B, T, Hq, Hkv, d, dp, topk, scale)
+
+
+def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False):
+    """Index Branch.  Returns (idx, nsel) or (idx, nsel, pooled_scores)."""
+    _bf16(qp, kp)
+    B, T, Hp, dp = qp.shape
+    dims = make_dims(B, T, Hp, Hp, 64, dp, topk)
+    idx = torch.empty((B, Hp, T, topk), dtype=torch.int32, device=qp.device)
+    nsel = torch.empty((B, Hp, T), dtype=torch.int32, device=qp.device)
+    nblk = (T + 127) // 128
+    pool = torch.empty((B, Hp, T, nblk), dtype=torch.float32, device=qp.device) if pooled else None
+    if ws is None:
+        ws = workspace(dims, MSA_SELECT, qp.device)
+    _check(LIB.msa_proxy_select(ctypes.byref(dims), _p(qp), _p(kp), _p(idx), _p(nsel), _p(pool), _p(ws),
+                                ws.numel(), _stream(stream)), "msa_proxy_select")
+    if check:
+        _check(check_status(ws, stream), "msa_proxy_select (device)")
+    return (idx, nsel, pool) if pooled else (idx, nsel)
+
+
+def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None):
+    """Main Branch forward.  Returns (o bf16 [B,T,Hq,d], lse fp32 [B,Hq,T])."""
+    _bf16(q, k, v)
+    B, T, Hq, d = q.shape
+    topk = idx.shape[3]
+    dims = make_dims(B, T, Hq, k.shape[2], d, 64, topk, scale)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    if ws is None:
+        ws = workspace(dims, MSA_FWD, q.device)
+    _check(LIB.msa_fwd(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(idx), _p(nsel), _p(o), _p(lse), _p(ws),
+                       ws.numel(), _stream(stream)), "msa_fwd")
+    if check:
+        _check(check_status(ws, stream), "msa_fwd (device)")
+    return o, lse
+
+
+def bwd(q, k, v, o, dout, lse, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None):
+    """Main Branch backward.  Returns (dq, dk, dv), bf16."""
+    _bf16(q, k, v, o, dout)
+    B, T, Hq, d = q.shape
+    topk = idx.shape[3]
+    dims = make_dims(B, T, Hq, k.shape[2], d, 64, topk, scale)
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    if ws is None:
+        ws = workspace(dims, MSA_BWD, q.device)
+    _check(LIB.msa_bwd(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(o), _p(dout), _p(lse), _p(idx),
+                       _p(nsel), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream)), "msa_bwd")
+    if check:
+        _check(check_status(ws, stream), "msa_bwd (device)")
+    return dq, dk, dv
+
+
+class MSAAttention(torch.autograd.Function):
+    """o = MSA(q, k, v; qp, kp, topk).  The block ids chosen in forward are
+    cached for backward; no gradient flows to qp/kp (the selection is
+    piecewise constant)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, qp, kp, topk, scale=0.0):
+        idx, nsel = proxy_select(qp, kp, topk)
+        o, lse = fwd(q, k, v, idx, nsel, scale)
+        ctx.save_for_backward(q, k, v, o, lse, idx, nsel)
+        ctx.scale = scale
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse, idx, nsel = ctx.saved_tensors
+        dq, dk, dv = bwd(q, k, v, o, dout.contiguous(), lse, idx, nsel, ctx.scale)
+        return dq, dk, dv, None, None, None, None
+
+
+def diag_umma(mode: int, A: torch.Tensor, B: torch.Tensor) -> torch.Tensor:
+    """One tcgen05 MMA D = A B^T with the given operand staging (see msa.h)."""
+    _bf16(A, B)
+    N, K = B.shape
+    D = torch.empty((128, N), dtype=torch.float32, device=A.device)
+    ws = torch.empty(256, dtype=torch.uint8, device=A.device)
+    _check(LIB.msa_diag_umma(mode, N, K, _p(A), _p(B), _p(D), _p(ws), _stream(None)), "msa_diag_umma")
+    return D
+
+
+def diag_wait_timeout(limit_ns: int, device="cuda") -> int:
+    ws = torch.zeros(256, dtype=torch.uint8, device=device)
+    return int(LIB.msa_diag_wait_timeout(limit_ns, _p(ws), _stream(None)))

@@ -1,0 +1,159 @@
+/*
+ * msa.h -- C ABI of libmsa.so, the B200 (sm_100a) training hot path of
+ * MiniMax Sparse Attention (MSA).
+ *
+ * The method (pages: "Flash-MSA: Open-Source Sparse Attention Kernels Debut",
+ * section "How MSA works"; the ai-beat news post on Flash-MSA training,
+ * paragraphs 1-4): an Index Branch scores every causal (query, key) pair with
+ * one small proxy head per GQA group, max-pools the scores over 128-key
+ * blocks and picks, per query, the blocks it will read; the picked block ids
+ * are cached.  A Main Branch then runs exact softmax attention (GQA) over
+ * only those blocks, forward and backward.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers, row-major, last index fastest,
+ *    16-byte aligned, owned by the caller.  bf16 tensors are passed as void*.
+ *  - Shapes:  q, o, dout, dq  [B][T][Hq][d]   bf16
+ *             k, v, dk, dv    [B][T][Hkv][d]  bf16
+ *             qp, kp          [B][T][Hp][dp]  bf16   (Hp == Hkv)
+ *             idx             [B][Hp][T][topk] int32, ascending, -1 padded
+ *             nsel            [B][Hp][T]       int32
+ *             lse             [B][Hq][T]       fp32 (natural-log logsumexp)
+ *  - `ws` is a caller-owned device workspace of at least
+ *    msa_workspace_size(dims, which) bytes (256-byte aligned).  Its content
+ *    on entry is irrelevant; the library keeps no state between calls.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued on it; no entry point synchronises or allocates.
+ *  - Arguments are validated before anything is enqueued; on an error code
+ *    nothing has been launched.  Kernels never trap: a device wait that
+ *    gives up or an index outside its range writes a status word inside `ws`,
+ *    which msa_check_status() reads.
+ *  - Limits: block == 128; Hq % Hkv == 0 with G = Hq/Hkv in {1,2,4,8,16};
+ *    d in {64,128}; dp a multiple of 8 in [8,64]; 1 <= topk <= 128;
+ *    0 <= T <= 2^20.  B == 0 or T == 0 is a valid empty call.
+ *  - Inputs must be finite.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct msa_dims {
+    int B;      /* batch                                                  */
+    int T;      /* sequence length (any value; the last block may be short) */
+    int Hq;     /* query heads                                            */
+    int Hkv;    /* key/value heads = GQA groups                           */
+    int Hp;     /* proxy heads, one per group: must equal Hkv             */
+    int d;      /* head dim of the Main Branch                            */
+    int dp;     /* head dim of the proxy head                             */
+    int block;  /* KV block length: must be 128                           */
+    int topk;   /* blocks read per query, own block included              */
+    float scale;/* softmax scale of the Main Branch; 0 -> 1/sqrt(d)       */
+} msa_dims;
+
+enum msa_status {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_DIMS = -1,  /* a size outside the limits above            */
+    MSA_ERR_NULL_PTR = -2,      /* a required pointer is NULL                 */
+    MSA_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned (ws: 256) */
+    MSA_ERR_WS_TOO_SMALL = -4,  /* ws_bytes < msa_workspace_size()            */
+    MSA_ERR_LAUNCH = -5,        /* a CUDA launch or async call failed         */
+    MSA_ERR_TIMEOUT = -6,       /* a bounded device wait gave up              */
+    MSA_ERR_DEVICE = -7,        /* current device is not sm_100               */
+    MSA_ERR_DRIVER = -8,        /* tensor-map encoding unavailable or failed  */
+    MSA_ERR_INDEX = -9          /* an idx entry outside its valid range       */
+};
+
+enum msa_phase { MSA_SELECT = 0, MSA_FWD = 1, MSA_BWD = 2 };
+
+/* Bytes of workspace `which` (an msa_phase) needs for these dims.
+ * Returns 0 for invalid dims. */
+MSA_API size_t msa_workspace_size(const msa_dims* dims, int which);
+
+/*
+ * Index Branch ("How MSA works": KVs selected in 128-key blocks by
+ * max-pooling proxy scores; one proxy head per group; indices cached).
+ *   score(b,g,i,j) = sum_c qp[b,i,g,c] * kp[b,j,g,c]        for j <= i
+ *   pooled(b,g,i,n) = max of score over the keys of block n (n <= i/128)
+ * Query i keeps its own block i/128 and the topk-1 best earlier blocks by
+ * pooled score, equal scores going to the lower block id; with at most topk
+ * eligible blocks it keeps them all.  idx rows are written ascending and
+ * padded with -1; nsel = number of valid entries.  Scores are accumulated in
+ * fp32 on the tensor cores and compared in fp32; the T x T score matrix
+ * never leaves the chip.
+ *   pooled_dbg: optional (NULL = off) [B][Hp][T][nblk] fp32 output of the
+ *   pooled scores, -inf past the query's own block; for tests, it costs an
+ *   extra write of B*Hp*T*nblk floats.
+ */
+MSA_API int msa_proxy_select(const msa_dims* dims, const void* qp, const void* kp, int32_t* idx,
+                     int32_t* nsel, float* pooled_dbg, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Main Branch forward (ai-beat post, paragraph 1: exact softmax attention
+ * over only the selected blocks; "How MSA works": GQA).  For every query
+ * head h of group g = h / (Hq/Hkv) and query i, the keys read are
+ * { j : j/128 in idx[b,g,i,:nsel], j <= i };
+ *   S_ij = scale * q_i . k_j,  L_i = log sum_j exp(S_ij),
+ *   O_i  = sum_j exp(S_ij - L_i) v_j.
+ * Writes o (bf16) and lse (fp32).  idx/nsel are the cached output of
+ * msa_proxy_select and must be valid (ascending, in range); entries outside
+ * [0, i/128] are reported as MSA_ERR_INDEX by msa_check_status.
+ */
+MSA_API int msa_fwd(const msa_dims* dims, const void* q, const void* k, const void* v, const int32_t* idx,
+            const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Main Branch backward (ai-beat post, paragraph 2: training needs custom
+ * backward kernels).  With P_ij = exp(S_ij - L_i) from the cached idx and
+ * lse, D_i = dout_i . o_i and dS_ij = P_ij (dout_i . v_j - D_i):
+ *   dq_i = scale sum_j dS_ij k_j,
+ *   dk_j = scale sum_{i,h in group} dS_ij q_i,  dv_j = sum_{i,h} P_ij dout_i.
+ * The block selection is piecewise constant: no gradient is produced for
+ * qp/kp.  Writes dq, dk, dv (bf16).
+ */
+MSA_API int msa_bwd(const msa_dims* dims, const void* q, const void* k, const void* v, const void* o,
+            const void* dout, const float* lse, const int32_t* idx, const int32_t* nsel, void* dq,
+            void* dk, void* dv, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the status word a previous call left in
+ * `ws`: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INDEX.  `code` (nullable)
+ * receives the raw device code (which wait or check failed). */
+MSA_API int msa_check_status(const void* ws, void* stream, uint32_t* code);
+
+/* Human-readable text for a status code (static storage). */
+MSA_API const char* msa_strerror(int status);
+
+/* ---- diagnostics (no counterpart on the pages; used by the GPU tests) ---- */
+
+/* One 128 x N x K tcgen05 MMA, D[m][n] = sum_k A[m][k] * B[n][k], with the
+ * operands staged the way the kernels stage them.  A: [128][K] bf16, B:
+ * [N][K] bf16, D: [128][N] fp32, all device pointers.  mode: 0 = A,B K-major
+ * in shared memory; 1 = A K-major, B MN-major; 2 = A,B MN-major; 3 = A in
+ * tensor memory, B MN-major; 4 = A in tensor memory, B K-major; adding 8
+ * exchanges the two byte offsets of the MN-major descriptors (a check that
+ * the convention in use is the right one).  N in {64,128}, K in {64,128};
+ * `ws` needs 256 bytes.  Synchronous. */
+MSA_API int msa_diag_umma(int mode, int N, int K, const void* A, const void* B, float* D, void* ws,
+                  void* stream);
+
+/* Launches a kernel whose mbarrier wait can never complete, bounded by
+ * limit_ns; returns what msa_check_status reports (MSA_ERR_TIMEOUT when the
+ * bound works).  `ws` needs 256 bytes.  Synchronous. */
+MSA_API int msa_diag_wait_timeout(uint64_t limit_ns, void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

@@ -66,6 +66,8 @@ def _load():
                                            P, P, ctypes.c_int]
         _lib.msa_oracle_bwd_dkdv.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, P, P, P, I64, P,
                                              P, P, ctypes.c_int]
+        _lib.msa_oracle_bwd_kv_rows.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, P, P, P, I64, P,
+                                                P, P, ctypes.c_int]
     return _lib
 
 
@@ -206,6 +208,26 @@ def bwd_dkdv(m: Dims, q, k, v, dout, lse, D, idx, nsel, blocks=None, dk=None, dv
     lib.msa_oracle_bwd_dkdv(ctypes.byref(dm), _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse),
                             _ptr(D), _ptr(idx), _ptr(nsel), len(bl), _ptr(bl), _ptr(dk), _ptr(dv),
                             _threads(nthreads))
+    return dk, dv
+
+
+def bwd_kv_rows(m: Dims, q, k, v, dout, lse, D, idx, nsel, rows, nthreads=None):
+    """Contributions of the listed query rows ((b*Hq+h)*T+i) to dK and dV of
+    each key the row reads, [nrows, topk*blk, d] each (keys in the row's
+    order, zero padded).  Needs the rows' L and D."""
+    lib = _load()
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    lse = np.ascontiguousarray(lse, dtype=np.float64)
+    D = np.ascontiguousarray(D, dtype=np.float64)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    nsel = np.ascontiguousarray(nsel, dtype=np.int32)
+    r = _rows(rows, m.B * m.Hq * m.T)
+    dk = np.empty((len(r), m.topk * m.blk, m.d), dtype=np.float64)
+    dv = np.empty((len(r), m.topk * m.blk, m.d), dtype=np.float64)
+    dm = m.c()
+    lib.msa_oracle_bwd_kv_rows(ctypes.byref(dm), _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse),
+                               _ptr(D), _ptr(idx), _ptr(nsel), len(r), _ptr(r), _ptr(dk), _ptr(dv),
+                               _threads(nthreads))
     return dk, dv
 
 

@@ -424,3 +424,61 @@ int msa_oracle_bwd_dkdv(const odims* m, const float* q, const float* k, const fl
     parallel_for(nblk_list, nthreads, kv_item, &c);
     return 0;
 }
+
+typedef struct {
+    const odims* m;
+    const float *q, *k, *v, *dout;
+    const double *lse, *D;
+    const int32_t *idx, *nsel;
+    const int64_t* rows;     /* flattened (b*Hq + h)*T + i */
+    double *dk, *dv;         /* per-row contributions, [nrows][blk*topk][d] */
+} kvr_ctx;
+
+static void kvr_item(void* vctx, int64_t r)
+{
+    kvr_ctx* c = (kvr_ctx*)vctx;
+    const odims* m = c->m;
+    const int T = m->T, d = m->d, G = m->Hq / m->Hkv;
+    int64_t row = c->rows[r];
+    int i = (int)(row % T);
+    int64_t bh = row / T;
+    int h = (int)(bh % m->Hq), b = (int)(bh / m->Hq), g = h / G;
+    int* keys = (int*)malloc(sizeof(int) * (size_t)(m->topk * m->blk + 1));
+    int nk = gather_keys(m, c->idx, c->nsel, b, g, i, keys);
+    const int64_t qoff = (((int64_t)b * T + i) * m->Hq + h) * d;
+    const double L = c->lse[((int64_t)b * m->Hq + h) * T + i];
+    const double Di = c->D[((int64_t)b * m->Hq + h) * T + i];
+    double* dkr = c->dk + r * (int64_t)m->topk * m->blk * d;
+    double* dvr = c->dv + r * (int64_t)m->topk * m->blk * d;
+    for (int t = 0; t < nk; ++t) {
+        const int64_t koff = (((int64_t)b * T + keys[t]) * m->Hkv + g) * d;
+        double sc = 0.0, dp = 0.0;
+        for (int e = 0; e < d; ++e) {
+            sc += (double)c->q[qoff + e] * (double)c->k[koff + e];
+            dp += (double)c->dout[qoff + e] * (double)c->v[koff + e];
+        }
+        double p = exp(m->scale * sc - L);
+        double ds = p * (dp - Di);
+        for (int e = 0; e < d; ++e) {
+            dvr[(int64_t)t * d + e] = p * (double)c->dout[qoff + e];
+            dkr[(int64_t)t * d + e] = m->scale * ds * (double)c->q[qoff + e];
+        }
+    }
+    for (int t = nk; t < m->topk * m->blk; ++t)
+        for (int e = 0; e < d; ++e) { dvr[(int64_t)t * d + e] = 0.0; dkr[(int64_t)t * d + e] = 0.0; }
+    free(keys);
+}
+
+/* What one query row (b, h, i) adds to dK and dV of each key it reads, in
+ * the order of the row's keys (selected blocks ascending, keys ascending).
+ * Output [nrows][topk*blk][d]; needs the row's L and D. */
+int msa_oracle_bwd_kv_rows(const odims* m, const float* q, const float* k, const float* v,
+                           const float* dout, const double* lse, const double* D,
+                           const int32_t* idx, const int32_t* nsel,
+                           int64_t nrows, const int64_t* rows, double* dk_rows, double* dv_rows,
+                           int nthreads)
+{
+    kvr_ctx c = {m, q, k, v, dout, lse, D, idx, nsel, rows, dk_rows, dv_rows};
+    parallel_for(nrows, nthreads, kvr_item, &c);
+    return 0;
+}

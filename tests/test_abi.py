@@ -1,0 +1,133 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/msa.h declares, sizes its workspaces, and rejects bad arguments
+before it would touch a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_09_b200 import build
+    build.build()
+    from block_sparse_attention_09_b200 import msa
+    return msa
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for required in ("msa_proxy_select", "msa_fwd", "msa_bwd", "msa_workspace_size", "msa_check_status",
+                     "msa_strerror"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (msa_[a-z_0-9]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    # nothing but the C ABI leaks out of the library
+    assert all(n.startswith("msa_") for n in exported)
+
+
+def test_strerror(lib):
+    assert lib.LIB.msa_strerror(0) == b"ok"
+    assert lib.LIB.msa_strerror(-6) == b"device wait timed out"
+    assert lib.LIB.msa_strerror(12345) == b"unknown status"
+
+
+def dims(lib, **kw):
+    base = dict(B=1, T=1024, Hq=4, Hkv=1, d=64, dp=32, topk=4)
+    base.update(kw)
+    return lib.make_dims(**base)
+
+
+def test_workspace_sizes(lib):
+    d = dims(lib)
+    sel = lib.workspace_size(d, lib.MSA_SELECT)
+    f = lib.workspace_size(d, lib.MSA_FWD)
+    b = lib.workspace_size(d, lib.MSA_BWD)
+    assert sel == 256
+    nblk, rows = 8, 1024 * 4
+    # index (count matrix, totals, pointers, token lists) + accumulators
+    assert f >= 256 + nblk * nblk * 4 + 1024 * 4 * 4 + rows * 64 * 4
+    assert b >= 256 + nblk * nblk * 4 + rows * 64 * 4
+    assert f % 256 == 0 and b % 256 == 0
+
+
+@pytest.mark.parametrize("bad", [dict(d=96), dict(dp=12), dict(dp=72), dict(topk=0), dict(topk=129),
+                                 dict(Hq=6, Hkv=4), dict(Hq=12, Hkv=4), dict(T=-1), dict(T=(1 << 20) + 1)])
+def test_invalid_dims_rejected(lib, bad):
+    d = dims(lib, **bad)
+    assert lib.workspace_size(d, lib.MSA_FWD) == 0
+    ws = ctypes.create_string_buffer(1 << 16)
+    rc = lib.LIB.msa_fwd(ctypes.byref(d), 16, 16, 16, 16, 16, 16, 16, ctypes.addressof(ws), 1 << 16, None)
+    assert rc == -1
+
+
+def test_block_must_be_128(lib):
+    d = dims(lib)
+    d.block = 64
+    assert lib.workspace_size(d, lib.MSA_SELECT) == 0
+
+
+def test_hp_must_equal_hkv(lib):
+    d = dims(lib)
+    d.Hp = 2
+    assert lib.workspace_size(d, lib.MSA_SELECT) == 0
+
+
+def aligned_buffer(nbytes, align=256):
+    raw = ctypes.create_string_buffer(nbytes + align)
+    addr = (ctypes.addressof(raw) + align - 1) & ~(align - 1)
+    return raw, addr
+
+
+def test_argument_errors_before_any_launch(lib):
+    d = dims(lib)
+    need = lib.workspace_size(d, lib.MSA_FWD)
+    raw, ws = aligned_buffer(64)
+    P = 4096  # an aligned non-null stand-in; never dereferenced on these paths
+    # workspace checks come first
+    assert lib.LIB.msa_fwd(ctypes.byref(d), P, P, P, P, P, P, P, None, need, None) == -2
+    assert lib.LIB.msa_fwd(ctypes.byref(d), P, P, P, P, P, P, P, ws + 16, need, None) == -3
+    assert lib.LIB.msa_fwd(ctypes.byref(d), P, P, P, P, P, P, P, ws, need - 1, None) == -4
+    # then tensor pointers
+    assert lib.LIB.msa_fwd(ctypes.byref(d), None, P, P, P, P, P, P, ws, need, None) == -2
+    assert lib.LIB.msa_fwd(ctypes.byref(d), P + 8, P, P, P, P, P, P, ws, need, None) == -3
+    nb = lib.workspace_size(d, lib.MSA_BWD)
+    assert lib.LIB.msa_bwd(ctypes.byref(d), P, P, P, P, P, P, P, P, P, P, None, ws, nb, None) == -2
+    assert lib.LIB.msa_proxy_select(ctypes.byref(d), P, P + 4, P, P, None, ws, 256, None) == -3
+
+
+def test_empty_problem_is_a_no_op(lib):
+    raw, ws = aligned_buffer(1 << 12)
+    for kw in (dict(T=0), dict(B=0)):
+        d = dims(lib, **kw)
+        need = lib.workspace_size(d, lib.MSA_FWD)
+        assert lib.LIB.msa_fwd(ctypes.byref(d), None, None, None, None, None, None, None, ws, need,
+                               None) == 0
+        assert lib.LIB.msa_proxy_select(ctypes.byref(d), None, None, None, None, None, ws, 256, None) == 0
+
+
+def test_no_gpu_reports_device_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    d = dims(lib)
+    raw, ws = aligned_buffer(256)
+    P = 4096
+    assert lib.LIB.msa_proxy_select(ctypes.byref(d), P, P, P, P, None, ws, 256, None) == -7

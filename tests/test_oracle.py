@@ -274,3 +274,27 @@ def test_bwd_block_subset_matches_all(oracle_mod):
         sl = slice(n * 128, (n + 1) * 128)
         assert np.array_equal(dk[0, sl, g], r["dk"][0, sl, g])
         assert np.array_equal(dv[0, sl, g], r["dv"][0, sl, g])
+
+
+def test_row_contributions_sum_to_block_gradients(oracle_mod):
+    """dK/dV built per KV block equal the sum of every query row's own
+    contributions (two different loop orders over the same definition)."""
+    m = Dims(B=1, T=300, Hq=4, Hkv=2, d=8, dp=8, topk=2)
+    x = rand_inputs(m, seed=66)
+    r = O.full(m, x["qp"], x["kp"], x["q"], x["k"], x["v"], x["dout"])
+    dkr, dvr = O.bwd_kv_rows(m, x["q"], x["k"], x["v"], x["dout"], r["lse"], r["D"], r["idx"],
+                             r["nsel"], rows=None)
+    dk = np.zeros_like(r["dk"])
+    dv = np.zeros_like(r["dv"])
+    for row in range(m.B * m.Hq * m.T):
+        i = row % m.T
+        h = (row // m.T) % m.Hq
+        b = row // (m.T * m.Hq)
+        g = h // m.G
+        keys = [j for n in r["idx"][b, g, i, :r["nsel"][b, g, i]] for j in range(n * 128, (n + 1) * 128)
+                if j <= i]
+        for t, j in enumerate(keys):
+            dk[b, j, g] += dkr[row, t]
+            dv[b, j, g] += dvr[row, t]
+    assert np.allclose(dk, r["dk"], atol=1e-12)
+    assert np.allclose(dv, r["dv"], atol=1e-12)
