@@ -1,0 +1,425 @@
+"""Benchmark of the MSA training hot path (Index Branch + Main Branch forward
+and backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 128k] [--impl ours|reference]
+
+One step = msa_proxy_select + msa_fwd + msa_bwd over one synthetic batch of
+the chosen workload, inputs resident in HBM.  Under torchrun every rank runs
+its own batch (seed = rank): the path shards by independent problems with no
+collective, so scaling is weak.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (the plain C implementation the
+tests check against) on a bounded sample of query rows of the same workload,
+on the host cores, and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MSA fwd+bwd TFLOP/s (selected-block FLOPs) and tokens/s at T=128K; % of bf16 peak"
+BLOCK = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="128k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0, help="query rows in the CPU sample (0 = auto)")
+    return ap.parse_args()
+
+
+def workload_name(cfg):
+    bias = {"none": "", "group": ", per-group low-rank proxy bias", "recency": ", planted local-recency proxy bias"}
+    return (f"MSA {cfg.name}: B={cfg.B} T={cfg.T} Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} dp={cfg.dp} "
+            f"topk={cfg.topk} (own block incl.), causal, fwd+bwd{bias[cfg.bias]}")
+
+
+# ---------------------------------------------------------------- FLOP model
+def flops_from_nsel(cfg, nsel_counts):
+    """Selected-block FLOPs of one batch.  pairs(i) = keys query i reads =
+    128 (nsel_i - 1) + (i mod 128) + 1 (other selected blocks whole, own block
+    up to i); forward 4 d per (query head, key) pair (QK^T and PV), backward
+    2.5x forward; proxy 2 dp per (query, key) pair over the key blocks the
+    selection actually scores (blocks before the query's own, for query
+    tiles with more eligible blocks than topk)."""
+    total_pairs = nsel_counts["pairs"]
+    f_fwd = 4.0 * cfg.d * cfg.G * total_pairs
+    f_bwd = 2.5 * f_fwd
+    f_proxy = 0.0
+    if cfg.topk > 1:
+        for qb in range((cfg.T + BLOCK - 1) // BLOCK):
+            if qb + 1 > cfg.topk:
+                rows = min(BLOCK, cfg.T - qb * BLOCK)
+                f_proxy += 2.0 * cfg.dp * rows * BLOCK * qb
+        f_proxy *= cfg.B * cfg.Hp
+    return f_proxy, f_fwd, f_bwd
+
+
+def pair_count(cfg, nsel):
+    import torch
+    i = torch.arange(cfg.T, device=nsel.device, dtype=torch.int64)
+    own = (i % BLOCK) + 1
+    pairs = BLOCK * (nsel.to(torch.int64) - 1) + own.view(1, 1, -1)
+    return {"pairs": float(pairs.sum().item())}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id):
+        self.device_id = device_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.device_id)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_arrays(host):
+    """float32 copies of the bf16 inputs (exact) for the oracle."""
+    return {k: v.float().numpy() for k, v in host.items()}
+
+
+def cpu_oracle_sample(cfg, x, rows_target, seed=0):
+    """Time the oracle on a bounded sample of query rows (b, g, i) of the
+    workload: selection (proxy scores of the row over all earlier keys, pool,
+    top-k), then forward, dQ and the row's dK/dV contributions for each of
+    the group's G heads.  Returns (credited FLOPs, seconds, rows, threads)."""
+    import oracle as O
+    from block_sparse_attention_09_b200.inputs import sample_rows
+    m = O.Dims(B=cfg.B, T=cfg.T, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, dp=cfg.dp, topk=cfg.topk)
+    threads = os.cpu_count() or 1
+    srows = sample_rows(cfg.B * cfg.Hkv * cfg.T, rows_target, seed=seed + 11)
+    t0 = time.perf_counter()
+    idx, nsel, _ = O.select(m, x["qp"], x["kp"], rows=srows, nthreads=threads)
+    qrows = []
+    for r in srows:
+        i = r % cfg.T
+        bg = r // cfg.T
+        b, g = divmod(bg, cfg.Hkv)
+        for hh in range(cfg.G):
+            qrows.append((b * cfg.Hq + g * cfg.G + hh) * cfg.T + i)
+    o, lse = O.fwd(m, x["q"], x["k"], x["v"], idx, nsel, rows=qrows, nthreads=threads)
+    dq, D = O.bwd_dq(m, x["q"], x["k"], x["v"], x["dout"], o, lse, idx, nsel, rows=qrows, nthreads=threads)
+    for c0 in range(0, len(qrows), 32):   # contributions are topk*128*d doubles per row: chunk them
+        O.bwd_kv_rows(m, x["q"], x["k"], x["v"], x["dout"], lse, D, idx, nsel, rows=qrows[c0:c0 + 32],
+                      nthreads=threads)
+    secs = time.perf_counter() - t0
+    flops = 0.0
+    for r in srows:
+        i = r % cfg.T
+        bg = r // cfg.T
+        b, g = divmod(bg, cfg.Hkv)
+        bi = i // BLOCK
+        ns = int(nsel[b, g, i])
+        pairs = BLOCK * (ns - 1) + (i % BLOCK) + 1
+        f_fwd = 4.0 * cfg.d * cfg.G * pairs
+        f_proxy = 2.0 * cfg.dp * BLOCK * bi if (bi + 1 > cfg.topk and cfg.topk > 1) else 0.0
+        flops += f_proxy + 3.5 * f_fwd
+    return flops, secs, len(srows), threads
+
+
+def calibrate_rows(cfg, x, seconds, cap=4096):
+    """Rows of the CPU sample that take about `seconds` on this host."""
+    fl, secs, n, _ = cpu_oracle_sample(cfg, x, 32, seed=99)
+    return max(8, min(cap, int(n * seconds / max(secs, 1e-3))))
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    from block_sparse_attention_09_b200.inputs import make_inputs
+    x = oracle_arrays(make_inputs(cfg, seed=0))
+    rows = args.cpu_rows or calibrate_rows(cfg, x, seconds=4.0)
+    vals = []
+    for s in range(args.warmup + args.steps):
+        fl, secs, n, threads = cpu_oracle_sample(cfg, x, rows, seed=s)
+        if s >= args.warmup:
+            vals.append((fl, secs))
+    fl = sum(v[0] for v in vals)
+    secs = sum(v[1] for v in vals)
+    value = fl / secs / 1e12
+    sample = f"{rows} query rows (b, group, i) per step, all {cfg.G} heads each, same workload and seeds"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(vals),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_name(cfg)},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    args = parse()
+    from block_sparse_attention_09_b200.inputs import CONFIGS, make_inputs
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
+    from block_sparse_attention_09_b200 import msa
+
+    # ---- inputs: seeded, generated on the host, one batch per rank
+    host = make_inputs(cfg, seed=rank)
+    host = {k: v.pin_memory() for k, v in host.items()}
+    d = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    torch.cuda.synchronize()
+    B, T, Hq, Hkv, D = cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.d
+    dims = msa.make_dims(B, T, Hq, Hkv, D, cfg.dp, cfg.topk)
+    ws_sel = msa.workspace(dims, msa.MSA_SELECT, dev)
+    ws_fwd = msa.workspace(dims, msa.MSA_FWD, dev)
+    ws_bwd = msa.workspace(dims, msa.MSA_BWD, dev)
+    o = torch.empty_like(d["q"])
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
+    stream = torch.cuda.current_stream()
+
+    def step(inputs, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        idx, nsel = msa.proxy_select(inputs["qp"], inputs["kp"], cfg.topk, ws=ws_sel)
+        if ev is not None:
+            ev[1].record(stream)
+        msa.fwd(inputs["q"], inputs["k"], inputs["v"], idx, nsel, ws=ws_fwd, out=(o, lse))
+        if ev is not None:
+            ev[2].record(stream)
+        msa.bwd(inputs["q"], inputs["k"], inputs["v"], o, inputs["dout"], lse, idx, nsel, ws=ws_bwd,
+                out=(dq, dk, dv))
+        if ev is not None:
+            ev[3].record(stream)
+        return idx, nsel
+
+    # correctness guard on the timed configuration: every device status word clean
+    idx, nsel = step(d)
+    for ws in (ws_sel, ws_fwd, ws_bwd):
+        rc = msa.check_status(ws)
+        if rc != 0:
+            raise RuntimeError(f"device status {rc} on the benchmark workload")
+    f_proxy, f_fwd, f_bwd = flops_from_nsel(cfg, pair_count(cfg, nsel))
+    f_step = f_proxy + f_fwd + f_bwd
+
+    for _ in range(args.warmup):
+        step(d)
+    torch.cuda.synchronize()
+
+    kernel_names = {msa.KERNEL_PROXY: "proxy_select", msa.KERNEL_FWD_MAIN: "fwd_main",
+                    msa.KERNEL_BWD_MAIN: "bwd_main"}
+    kev = {k: [] for k in kernel_names}
+    pev = []
+    try:
+        gpu_id = str(torch.cuda.get_device_properties(local).uuid)
+        gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
+    except Exception:
+        gpu_id = str(local)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        for kk in kernel_names:
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            kev[kk].append((a, b_))
+            msa.set_kernel_events(kk, a, b_)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        pev.append(ev)
+        step(d, ev)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    for kk in kernel_names:
+        msa.set_kernel_events(kk, None, None)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_stop) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    phase = {"proxy_select": [], "fwd": [], "bwd": []}
+    for ev in pev:
+        phase["proxy_select"].append(ev[0].elapsed_time(ev[1]))
+        phase["fwd"].append(ev[1].elapsed_time(ev[2]))
+        phase["bwd"].append(ev[2].elapsed_time(ev[3]))
+    phase_ms = {k: statistics.mean(v) for k, v in phase.items()}
+    kern_ms = {kernel_names[k]: statistics.mean(a.elapsed_time(b_) for a, b_ in v) for k, v in kev.items()}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        out_host = {"o": torch.empty_like(o, device="cpu").pin_memory(),
+                    "dq": torch.empty_like(dq, device="cpu").pin_memory(),
+                    "dk": torch.empty_like(dk, device="cpu").pin_memory(),
+                    "dv": torch.empty_like(dv, device="cpu").pin_memory()}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+        e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            for k, v in host.items():      # this step's inputs from pinned host memory
+                d[k].copy_(v, non_blocking=True)
+            step(d)
+            out_host["o"].copy_(o, non_blocking=True)
+            out_host["dq"].copy_(dq, non_blocking=True)
+            out_host["dk"].copy_(dk, non_blocking=True)
+            out_host["dv"].copy_(dv, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b_) / e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * f_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = measured_peaks()
+    tflops = world * f_step / (ms * 1e-3) / 1e12
+    tok_s = world * B * T / (ms * 1e-3)
+    # dominant kernel of the step
+    kf = {"proxy_select": f_proxy, "fwd_main": f_fwd, "bwd_main": f_bwd}
+    dom = max(kern_ms, key=lambda k: kern_ms[k])
+    achieved = kf[dom] / (kern_ms[dom] * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None,
+            "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+            "frac_of_burst": achieved / float(peaks.get("bf16_tflops", peak))}
+
+    cpu = None
+    if not args.no_cpu and world == 1:
+        x = oracle_arrays(host)
+        rows = args.cpu_rows or calibrate_rows(cfg, x, seconds=15.0)
+        fl, secs, n, threads = cpu_oracle_sample(cfg, x, rows, seed=0)
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} query rows (b, group, i) of the same workload, all {cfg.G} heads each: "
+                         f"selection, forward, dQ and dK/dV contributions; {secs:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 inputs" + (", planted local-recency proxy bias" if cfg.bias == "recency" else ""),
+        "config": {"workload": workload_name(cfg), "B": B, "T": T, "Hq": Hq, "Hkv": Hkv, "d": D,
+                   "dp": cfg.dp, "topk": cfg.topk, "per_rank": "one batch per rank (seed = rank)",
+                   "l2": "inputs larger than L2 (Q alone %.2f GB), no flush" % (d["q"].numel() * 2 / 1e9)},
+        "tokens_per_s": tok_s,
+        "frac_of_peak": tflops / float(peaks.get("bf16_tflops")),
+        "flops_per_step": {"proxy": f_proxy, "fwd": f_fwd, "bwd": f_bwd},
+        "phases_ms": phase_ms,
+        "phase_tflops": {"proxy_select": f_proxy / (phase_ms["proxy_select"] * 1e-3) / 1e12,
+                         "fwd": f_fwd / (phase_ms["fwd"] * 1e-3) / 1e12,
+                         "bwd": f_bwd / (phase_ms["bwd"] * 1e-3) / 1e12,
+                         "fwd+bwd": (f_fwd + f_bwd) / ((phase_ms["fwd"] + phase_ms["bwd"]) * 1e-3) / 1e12},
+        "kernel_ms": kern_ms,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 16 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

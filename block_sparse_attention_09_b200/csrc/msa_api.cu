@@ -74,6 +74,12 @@ bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t e0, uint64_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+TraceEvents& trace_events()
+{
+    static thread_local TraceEvents t;
+    return t;
+}
+
 }  // namespace msa
 
 using namespace msa;
@@ -240,6 +246,15 @@ const char* msa_strerror(int s)
     case MSA_ERR_INDEX: return "block index out of range";
     default: return "unknown status";
     }
+}
+
+int msa_set_kernel_events(int kernel, void* start, void* stop)
+{
+    if (kernel < 0 || kernel >= kTraceCount) return MSA_ERR_INVALID_DIMS;
+    TraceEvents& t = trace_events();
+    t.start[kernel] = (cudaEvent_t)start;
+    t.stop[kernel] = (cudaEvent_t)stop;
+    return MSA_OK;
 }
 
 int msa_diag_umma(int mode, int N, int K, const void* A, const void* B, float* D, void* ws, void* stream)

@@ -42,6 +42,24 @@ WsLayout ws_layout(const Problem& p, int which);
 bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t e0, uint64_t e1, uint64_t e2,
                        uint64_t e3, uint32_t box0, uint32_t box2);
 
+// ---- tracing: CUDA events recorded around the main kernels ---------------
+enum TraceKernel : int { kTraceProxy = 0, kTraceFwdMain = 1, kTraceBwdMain = 2, kTraceCount = 3 };
+struct TraceEvents {
+    cudaEvent_t start[kTraceCount] = {nullptr, nullptr, nullptr};
+    cudaEvent_t stop[kTraceCount] = {nullptr, nullptr, nullptr};
+};
+TraceEvents& trace_events();   // per host thread
+inline void trace_begin(int k, cudaStream_t st)
+{
+    TraceEvents& t = trace_events();
+    if (t.start[k]) cudaEventRecord(t.start[k], st);
+}
+inline void trace_end(int k, cudaStream_t st)
+{
+    TraceEvents& t = trace_events();
+    if (t.stop[k]) cudaEventRecord(t.stop[k], st);
+}
+
 // ---- launchers (return cudaGetLastError() of their launches) -------------
 cudaError_t launch_proxy_select(const Problem& p, const CUtensorMap& tm_qp, const CUtensorMap& tm_kp,
                                 int32_t* idx, int32_t* nsel, float* pooled, uint32_t* status,

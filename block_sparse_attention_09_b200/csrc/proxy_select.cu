@@ -283,7 +283,9 @@ cudaError_t launch_proxy_select(const Problem& pr, const CUtensorMap& tm_qp, con
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(pr.nblk * pr.B * pr.Hp);
+    trace_begin(kTraceProxy, st);
     proxy_select_kernel<<<grid, kThreads, smem, st>>>(tm_qp, tm_kp, p);
+    trace_end(kTraceProxy, st);
     return cudaGetLastError();
 }
 

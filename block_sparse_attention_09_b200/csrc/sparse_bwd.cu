@@ -445,7 +445,9 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
+    trace_begin(kTraceBwdMain, st);
     bwd_main_kernel<D><<<(unsigned)(pr.nblk * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+    trace_end(kTraceBwdMain, st);
     const int64_t n8 = pr.rows_q() * D / 8;
     bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dqacc, (__nv_bfloat16*)dq, n8);
     return cudaGetLastError();

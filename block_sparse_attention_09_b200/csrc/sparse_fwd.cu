@@ -472,7 +472,9 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     if ((e = cudaFuncSetAttribute(fwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
+    trace_begin(kTraceFwdMain, st);
     fwd_main_kernel<D><<<(unsigned)(pr.nblk * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+    trace_end(kTraceFwdMain, st);
 
     const int64_t fth = (int64_t)pr.rows_q() * (D / 8);
     fwd_finalize_kernel<D><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(

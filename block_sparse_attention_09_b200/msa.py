@@ -59,8 +59,9 @@ def _load():
     lib.msa_strerror.restype = ctypes.c_char_p
     lib.msa_diag_umma.argtypes = [I, I, I, P, P, P, P, P]
     lib.msa_diag_wait_timeout.argtypes = [U64, P, P]
+    lib.msa_set_kernel_events.argtypes = [I, P, P]
     for f in ("msa_proxy_select", "msa_fwd", "msa_bwd", "msa_check_status", "msa_diag_umma",
-              "msa_diag_wait_timeout"):
+              "msa_diag_wait_timeout", "msa_set_kernel_events"):
         getattr(lib, f).restype = I
     return lib
 
@@ -189,6 +190,17 @@ class MSAAttention(torch.autograd.Function):
         q, k, v, o, lse, idx, nsel = ctx.saved_tensors
         dq, dk, dv = bwd(q, k, v, o, dout.contiguous(), lse, idx, nsel, ctx.scale)
         return dq, dk, dv, None, None, None, None
+
+
+KERNEL_PROXY, KERNEL_FWD_MAIN, KERNEL_BWD_MAIN = 0, 1, 2
+
+
+def set_kernel_events(kernel: int, start=None, stop=None) -> None:
+    """Record torch.cuda.Event ``start``/``stop`` around the named kernel in
+    later calls from this thread (None stops recording)."""
+    s = ctypes.c_void_p(start.cuda_event) if start is not None else None
+    e = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
+    _check(LIB.msa_set_kernel_events(kernel, s, e), "msa_set_kernel_events")
 
 
 def diag_umma(mode: int, A: torch.Tensor, B: torch.Tensor) -> torch.Tensor:

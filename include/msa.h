@@ -134,6 +134,16 @@ MSA_API int msa_check_status(const void* ws, void* stream, uint32_t* code);
 /* Human-readable text for a status code (static storage). */
 MSA_API const char* msa_strerror(int status);
 
+/* ---- tracing (no counterpart on the pages) -------------------------------- */
+
+enum msa_kernel { MSA_KERNEL_PROXY = 0, MSA_KERNEL_FWD_MAIN = 1, MSA_KERNEL_BWD_MAIN = 2 };
+
+/* From now on, calls made by this host thread record the CUDA event `start`
+ * (a cudaEvent_t) on the call's stream just before launching the named
+ * kernel, and `stop` just after it, so a caller can time that kernel alone.
+ * NULL stops recording.  The events stay owned by the caller. */
+MSA_API int msa_set_kernel_events(int kernel, void* start, void* stop);
+
 /* ---- diagnostics (no counterpart on the pages; used by the GPU tests) ---- */
 
 /* One 128 x N x K tcgen05 MMA, D[m][n] = sum_k A[m][k] * B[n][k], with the
