@@ -302,6 +302,8 @@ def main():
     for _ in range(args.steps):
         for kk in kernel_names:
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)      # torch creates the CUDA event on first record;
+            b_.record(stream)     # the library records it again around the kernel
             kev[kk].append((a, b_))
             msa.set_kernel_events(kk, a, b_)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
