@@ -216,3 +216,24 @@ def diag_umma(mode: int, A: torch.Tensor, B: torch.Tensor) -> torch.Tensor:
 def diag_wait_timeout(limit_ns: int, device="cuda") -> int:
     ws = torch.zeros(256, dtype=torch.uint8, device=device)
     return int(LIB.msa_diag_wait_timeout(limit_ns, _p(ws), _stream(None)))
+
+
+def fwd_noalloc(q, k, v, idx, nsel, scale=0.0, stream=None, out=None):
+    """msa_fwd_noalloc: the forward with the library's fixed 64 MiB device
+    scratch instead of a caller workspace, for callers that cannot allocate
+    device memory.  Only problems whose forward workspace fits 64 MiB; calls
+    that overlap on the GPU must be serialised (they share the scratch)."""
+    fn = LIB.msa_fwd_noalloc
+    fn.argtypes = [ctypes.POINTER(Dims)] + [ctypes.c_void_p] * 8
+    fn.restype = ctypes.c_int
+    _bf16(q, k, v)
+    B, T, Hq, d = q.shape
+    dims = make_dims(B, T, Hq, k.shape[2], d, 64, idx.shape[3], scale)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    _check(fn(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(idx), _p(nsel), _p(o), _p(lse), _stream(stream)),
+           "msa_fwd_noalloc")
+    return o, lse

@@ -126,6 +126,30 @@ MSA_API int msa_bwd(const msa_dims* dims, const void* q, const void* k, const vo
             const void* dout, const float* lse, const int32_t* idx, const int32_t* nsel, void* dq,
             void* dk, void* dv, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * msa_fwd without a workspace argument (the pages have no counterpart: this
+ * is a library convenience).  For callers that cannot allocate device
+ * memory or hand over a workspace -- a plugin or custom-op host that owns all
+ * device memory through its own pool and gives an operator only its inputs
+ * and outputs, or a latency-critical loop where cudaMalloc/cudaFree (which
+ * can synchronise the device) is not allowed.  Same arguments, layouts and
+ * results as msa_fwd; the workspace is a fixed 64 MiB array inside the
+ * library that every GPU loading this part of the library keeps until the
+ * process exits.  The call allocates nothing.
+ *  - Problems whose forward workspace (msa_workspace_size(dims, MSA_FWD))
+ *    exceeds 64 MiB are rejected with MSA_ERR_WS_TOO_SMALL before any launch.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents (whatever must start at zero is cleared by every call).  Calls
+ *    whose work overlaps on the GPU race on it: serialise them.
+ *  - Device-side status (timeouts, malformed idx) stays in the shared array
+ *    and is not reported; validate idx with msa_fwd when in doubt.
+ */
+MSA_API int msa_fwd_noalloc(const msa_dims* dims, const void* q, const void* k, const void* v,
+                            const int32_t* idx, const int32_t* nsel, void* o, float* lse, void* stream);
+
 /* Synchronises `stream`, then reads the status word a previous call left in
  * `ws`: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INDEX.  `code` (nullable)
  * receives the raw device code (which wait or check failed). */
