@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="query rows in the CPU sample (0 = auto)")
+    ap.add_argument("--bias", default=None, choices=["none", "group", "recency"],
+                    help="override the workload's proxy-input structure (profiling variants)")
     return ap.parse_args()
 
 
@@ -221,6 +223,8 @@ def main():
     args = parse()
     from block_sparse_attention_09_b200.inputs import CONFIGS, make_inputs
     cfg = CONFIGS[args.config]
+    if args.bias is not None:
+        cfg = cfg.with_(bias=args.bias)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -36,6 +36,8 @@ WsLayout ws_layout(const Problem& p, int which)
     if (which == MSA_BWD) {
         L.dsum = take(rows * 4);
         L.dqacc = take(rows * p.d * 4);
+        L.dkacc = take((size_t)p.B * p.T * p.Hkv * p.d * 4);
+        L.dvacc = take((size_t)p.B * p.T * p.Hkv * p.d * 4);
     }
     L.total = off;
     return L;

@@ -267,6 +267,48 @@ MSA_DEV uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col)
     return base + (lane << 16) + col;
 }
 
+// ---------------------------------------------------------------- work items
+// The Main Branch kernels walk (group, query range, KV block) items: all KV
+// blocks n that queries of range R (RB query blocks) may read, group by
+// group and range by range, so the query-side rows they gather from and
+// reduce into stay in L2 while a range is processed.  The token segment of
+// an item comes from the inverse index: ptr[bg][n] starts block n's list and
+// off[bg][qb][n] (valid for qb >= n) counts its tokens in query blocks
+// before qb.
+struct RangeItem {
+    int bg, n, beg, count;   // beg: offset into the group's token list
+};
+
+__host__ __device__ inline int range_items_per_group(int nblk, int RB)
+{
+    int total = 0;
+    for (int R = 0; R * RB < nblk; ++R) total += min(nblk, (R + 1) * RB);
+    return total;
+}
+
+MSA_DEV RangeItem range_item(int x, int nblk, int RB, int per_group, const int32_t* ptr, const int32_t* off)
+{
+    RangeItem it;
+    it.bg = x / per_group;
+    int rem = x % per_group, R = 0;
+    for (;;) {
+        const int nv = min(nblk, (R + 1) * RB);
+        if (rem < nv) break;
+        rem -= nv;
+        ++R;
+    }
+    const int n = rem, qs = R * RB, qe = min(nblk, (R + 1) * RB);
+    const int32_t* pp = ptr + (int64_t)it.bg * (nblk + 1);
+    const int32_t* o = off + (int64_t)it.bg * nblk * nblk;
+    const int base = pp[n];
+    const int start = qs > n ? o[(int64_t)qs * nblk + n] : 0;
+    const int end = qe >= nblk ? pp[n + 1] - base : o[(int64_t)qe * nblk + n];
+    it.n = n;
+    it.beg = base + start;
+    it.count = end - start;
+    return it;
+}
+
 // ---------------------------------------------------------------- math
 MSA_DEV float fmax3(float a, float b, float c)
 {

@@ -32,7 +32,7 @@ struct WsLayout {
     size_t status = 0;                           // 256 B: status word, index-error word
     size_t cnt = 0, tot = 0, ptr = 0, tok = 0;   // block -> query inverse index
     size_t qnorm = 0, kmax = 0, oacc = 0, lacc = 0, nflag = 0, flags = 0;   // forward
-    size_t dsum = 0, dqacc = 0;                  // backward
+    size_t dsum = 0, dqacc = 0, dkacc = 0, dvacc = 0;   // backward
     size_t total = 0;
 };
 WsLayout ws_layout(const Problem& p, int which);
@@ -41,6 +41,18 @@ WsLayout ws_layout(const Problem& p, int which);
 // box and 128-byte swizzle.  Returns false if the driver refused it.
 bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t e0, uint64_t e1, uint64_t e2,
                        uint64_t e3, uint32_t box0, uint32_t box2);
+
+// Query blocks per work-item range of the Main Branch kernels: the query-side
+// rows one range touches (fp32 accumulators and gathered bf16 inputs of a
+// group) stay near 24 MB, well inside L2.
+inline int range_blocks(const Problem& p)
+{
+    const long bytes_per_block = 128L * p.G * p.d * (4 + 2);
+    long rb = (24L << 20) / bytes_per_block;
+    if (rb < 1) rb = 1;
+    if (rb > p.nblk) rb = p.nblk;
+    return (int)rb;
+}
 
 // ---- tracing: CUDA events recorded around the main kernels ---------------
 enum TraceKernel : int { kTraceProxy = 0, kTraceFwdMain = 1, kTraceBwdMain = 2, kTraceCount = 3 };

@@ -32,6 +32,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdParams {
     int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
+    int RB, per_group;   // query blocks per range; work items per (b, group)
     float c1;      // scale * log2(e)
     float scale;
     const __nv_bfloat16* q;
@@ -39,10 +40,11 @@ struct BwdParams {
     const float* lse;
     const float* dsum;
     const int32_t* ptr;
+    const int32_t* off;
     const int32_t* tok;
     float* dqacc;
-    __nv_bfloat16* dk;
-    __nv_bfloat16* dv;
+    float* dkacc;    // fp32 dK, dV accumulators [B][T][Hkv][D]: one partial per item
+    float* dvacc;
     uint32_t* status;
 };
 
@@ -70,32 +72,18 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = p.B * p.Hkv;
-    const int n = (int)(blockIdx.x / BH), bg = (int)(blockIdx.x % BH);
+    const RangeItem item = range_item((int)blockIdx.x, p.nblk, p.RB, p.per_group, p.ptr, p.off);
+    const int n = item.n, bg = item.bg;
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int G = 1 << p.lgG;
-    const int32_t* pp = p.ptr + (int64_t)bg * (p.nblk + 1);
-    const int beg = pp[n];
-    const int count = pp[n + 1] - beg;
+    const int count = item.count;
     const uint32_t code0 = kStTimeoutBase + kKidBwd * 16;
-
-    if (count <= 0) {
-        // no query reads this block: its dK, dV are zero
-        const int rows = min(128, p.T - n * 128);
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        for (int x = threadIdx.x; x < rows * (D / 8); x += blockDim.x) {
-            const int j = n * 128 + x / (D / 8), e = (x % (D / 8)) * 8;
-            const int64_t off = (((int64_t)b * p.T + j) * p.Hkv + g) * D + e;
-            *reinterpret_cast<uint4*>(p.dk + off) = z;
-            *reinterpret_cast<uint4*>(p.dv + off) = z;
-        }
-        return;
-    }
+    if (count <= 0) return;   // accumulators start at zero: nothing to add
     if ((smem_u32(smem) & 1023u) != 0u) {   // the swizzled tiles need a 1024-byte aligned base
         if (threadIdx.x == 0) atomicCAS(p.status, 0u, code0 + 15);
         return;
     }
-    const int32_t* toks = p.tok + (int64_t)bg * p.T * p.topk + beg;
+    const int32_t* toks = p.tok + (int64_t)bg * p.T * p.topk + item.beg;
     const int nchunks = (count + p.tpc - 1) / p.tpc;
 
     uint8_t* k_tile = smem + SM::kK;
@@ -159,7 +147,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) {
             constexpr uint32_t idSS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
             constexpr uint32_t idKV = idesc_bf16(128, D, false, true);      // dV, dK (A in TMEM)
-            constexpr uint32_t idQ = idesc_bf16(128, D, true, true);        // dQ
+            constexpr uint32_t idQ = idesc_bf16(128, D, true, true);        // dQ (d = 64)
+            constexpr uint32_t idQT = idesc_bf16(128, 128, true, true);     // dQ^T (d = 128)
             const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile), dsa = smem_u32(ds_tile);
             bool ok = mbar_wait(kv_full, 0, wc, code0 + 0);
             for (int c = 0; ok && c < nchunks; ++c) {
@@ -188,11 +177,22 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 for (int kk = 0; kk < 8; ++kk)
                     umma_ts(tdK, tdP + kk * 8, desc_mnmajor(qa, 128, kk * 16), idKV,
                             (c > 0 || kk > 0) ? 1u : 0u);
+                if constexpr (D == 128) {
+                    // dQ^T = K^T dS^T: one TMEM lane per head-dim index, so the
+                    // epilogue's reductions cover whole cache lines
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ss(tdP, desc_mnmajor(dsa, 128, kk * 16), desc_mnmajor(ka, 128, kk * 16), idQ,
-                            kk > 0 ? 1u : 0u);
-                umma_commit(&st_empty[s]);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ss(tdP, desc_mnmajor(ka, 128, kk * 16), desc_mnmajor(dsa, 128, kk * 16), idQT,
+                                kk > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ss(tdP, desc_mnmajor(dsa, 128, kk * 16), desc_mnmajor(ka, 128, kk * 16), idQ,
+                                kk > 0 ? 1u : 0u);
+                }
+                // d = 128: the dQ epilogue stages through this chunk's Q/dO buffers
+                // and releases them itself once its bulk reductions have read them
+                if constexpr (D != 128) umma_commit(&st_empty[s]);
                 umma_commit(ds_empty);
                 umma_commit(dq_full);
             }
@@ -293,31 +293,70 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_arrive(p_full);
         }
     } else {
-        // ---------------- dQ partials out; dK, dV at the end ----------------
-        const int r = ((warp & 3) << 5) | lane;
+        // ---------------- dQ partials out; dK, dV partials at the end ----------------
+        const int r = ((warp & 3) << 5) | lane;    // TMEM lane of this thread
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
             ok = mbar_wait(dq_full, (uint32_t)c & 1u, wc, code0 + 7);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            const int jj = c * p.tpc + t;
-            const bool valid = jj < count;
-            const int i = valid ? toks[jj] : 0;
-            float* dst = p.dqacc + (((int64_t)b * p.T + i) * p.Hq + h) * D;
             const uint32_t ta = tmem_addr(tdP, lane_base, 0);
+            const int ntok = min(p.tpc, count - c * p.tpc);
+            if constexpr (D == 128) {
+                // lane r holds dQ^T[r][row] for the chunk's 128 rows.  Stage them
+                // row-major ([row][d], the global order of a token's G heads) in
+                // this chunk's Q/dO buffers -- every store of a row is 32
+                // consecutive floats, no bank conflicts -- then reduce each token's
+                // G*D floats with one bulk operation.
+                const int s = c & 1;
+                const uint32_t stg = smem_u32(q_stage(s));
 #pragma unroll
-            for (int piece = 0; piece < D / 32; ++piece) {
-                uint32_t v[32];
-                tmem_ld32(ta + piece * 32, v);
-                tmem_ld_wait();
-                if (valid) {
+                for (int piece = 0; piece < 4; ++piece) {
+                    uint32_t v[32];
+                    tmem_ld32(ta + piece * 32, v);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        red_add_v4(dst + piece * 32 + 4 * e, __uint_as_float(v[4 * e]),
-                                   __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
-                                   __uint_as_float(v[4 * e + 3]));
+                    for (int e = 0; e < 32; ++e)
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + ((piece * 32 + e) * D + r) * 4),
+                                     "r"(v[e])
+                                     : "memory");
+                }
+                tc_fence_before();
+                mbar_arrive(dq_empty);
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                const int tid = threadIdx.x - 320;
+                const uint32_t tok_bytes = (uint32_t)G * D * 4u;
+                for (int t = tid; t < ntok; t += 128) {
+                    const int i = toks[c * p.tpc + t];
+                    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                                     p.dqacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D),
+                                 "r"(stg + (uint32_t)t * tok_bytes), "r"(tok_bytes)
+                                 : "memory");
+                }
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                named_bar_sync(1, 128);
+                if (tid == 0) mbar_arrive(&st_empty[s]);
+                continue;
+            } else {
+                const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
+                const bool valid = t < ntok;
+                const int i = valid ? toks[c * p.tpc + t] : 0;
+                float* dst = p.dqacc + (((int64_t)b * p.T + i) * p.Hq + h) * D;
+#pragma unroll
+                for (int piece = 0; piece < D / 32; ++piece) {
+                    uint32_t v[32];
+                    tmem_ld32(ta + piece * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            red_add_v4(dst + piece * 32 + 4 * e, __uint_as_float(v[4 * e]),
+                                       __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
+                                       __uint_as_float(v[4 * e + 3]));
+                    }
                 }
             }
             tc_fence_before();
@@ -325,30 +364,41 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         if (ok) ok = mbar_wait(kv_done, 0, wc, code0 + 8);
         if (__all_sync(0xffffffffu, ok)) {
+            // This item's dK, dV partials (lane = key) -> padded staging in the
+            // now idle Q/dO stages -> one bulk fp32 reduction per key row.
             tc_fence_after();
+            const uint32_t row_stride = D * 4u + 16u;
+            const uint32_t stg = smem_u32(smem + SM::kStage0);
             const int j = n * 128 + r;   // this lane's key
-            const int64_t off = (((int64_t)b * p.T + j) * p.Hkv + g) * D;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const uint32_t ta = tmem_addr(which == 0 ? tdV : tdK, lane_base, 0);
-                __nv_bfloat16* out = (which == 0 ? p.dv : p.dk) + off;
+                const uint32_t row = stg + (uint32_t)which * 128u * row_stride + (uint32_t)r * row_stride;
 #pragma unroll
                 for (int piece = 0; piece < D / 32; ++piece) {
                     uint32_t v[32];
                     tmem_ld32(ta + piece * 32, v);
                     tmem_ld_wait();
-                    if (j < p.T) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            uint4 u;
-                            u.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]), __uint_as_float(v[8 * e + 1]));
-                            u.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3]));
-                            u.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5]));
-                            u.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7]));
-                            *reinterpret_cast<uint4*>(out + piece * 32 + 8 * e) = u;
-                        }
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (piece * 32 + 4 * e) * 4),
+                                     "r"(v[4 * e]), "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3])
+                                     : "memory");
                 }
+            }
+            fence_proxy_async_smem();
+            if (j < p.T) {
+                const int64_t off = (((int64_t)b * p.T + j) * p.Hkv + g) * D;
+#pragma unroll
+                for (int which = 0; which < 2; ++which) {
+                    float* dst = (which == 0 ? p.dvacc : p.dkacc) + off;
+                    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+                                 "r"(stg + (uint32_t)which * 128u * row_stride + (uint32_t)r * row_stride),
+                                 "r"((uint32_t)D * 4u)
+                                 : "memory");
+                }
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
             }
         }
     }
@@ -418,9 +468,14 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     uint8_t* w = (uint8_t*)ws;
     float* dsum = (float*)(w + L.dsum);
     float* dqacc = (float*)(w + L.dqacc);
+    float* dkacc = (float*)(w + L.dkacc);
+    float* dvacc = (float*)(w + L.dvacc);
+    const size_t kv_elems = (size_t)pr.B * pr.T * pr.Hkv * D;
     cudaError_t e;
     if ((e = cudaMemsetAsync(dqacc, 0, sizeof(float) * (size_t)pr.rows_q() * D, st)) != cudaSuccess)
         return e;
+    if ((e = cudaMemsetAsync(dkacc, 0, sizeof(float) * kv_elems, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dvacc, 0, sizeof(float) * kv_elems, st)) != cudaSuccess) return e;
     const int64_t th = pr.rows_q() * (D / 8);
     bwd_dsum_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(
         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, dsum);
@@ -436,20 +491,26 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     p.lse = lse;
     p.dsum = dsum;
     p.ptr = (const int32_t*)(w + L.ptr);
+    p.off = (const int32_t*)(w + L.cnt);
     p.tok = (const int32_t*)(w + L.tok);
     p.dqacc = dqacc;
-    p.dk = (__nv_bfloat16*)dk;
-    p.dv = (__nv_bfloat16*)dv;
+    p.dkacc = dkacc;
+    p.dvacc = dvacc;
     p.status = (uint32_t*)(w + L.status);
+    p.RB = range_blocks(pr);
+    p.per_group = range_items_per_group(pr.nblk, p.RB);
     const size_t smem = BwdSmem<D>::kTotal;
     if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
     trace_begin(kTraceBwdMain, st);
-    bwd_main_kernel<D><<<(unsigned)(pr.nblk * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+    bwd_main_kernel<D><<<(unsigned)(p.per_group * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
     trace_end(kTraceBwdMain, st);
     const int64_t n8 = pr.rows_q() * D / 8;
     bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dqacc, (__nv_bfloat16*)dq, n8);
+    const int64_t k8 = (int64_t)kv_elems / 8;
+    bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dkacc, (__nv_bfloat16*)dk, k8);
+    bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dvacc, (__nv_bfloat16*)dv, k8);
     return cudaGetLastError();
 }
 

@@ -36,10 +36,12 @@ constexpr float kUnderflow = 5.421010862427522e-20f;   // 2^-64: row sums below 
 
 struct FwdParams {
     int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
+    int RB, per_group;   // query blocks per range; work items per (b, group)
     float c1;        // scale * log2(e)
     float bound;     // |scale| * log2(e)
     const __nv_bfloat16* q;
     const int32_t* ptr;
+    const int32_t* off;
     const int32_t* tok;
     const float* qn;
     const float* kmax;
@@ -55,25 +57,32 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 {
     constexpr uint32_t kTile = 128u * D * 2u;   // 128 rows x D bf16
     constexpr int kSlabs = D / 64;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = p.B * p.Hkv;
-    const int n = (int)(blockIdx.x / BH), bg = (int)(blockIdx.x % BH);   // low blocks (most selected) first
+    const RangeItem item = range_item((int)blockIdx.x, p.nblk, p.RB, p.per_group, p.ptr, p.off);
+    const int n = item.n, bg = item.bg;
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int G = 1 << p.lgG;
-    const int32_t* pp = p.ptr + (int64_t)bg * (p.nblk + 1);
-    const int beg = pp[n];
-    const int count = pp[n + 1] - beg;
+    const int count = item.count;
     if (count <= 0) return;
-    const int32_t* toks = p.tok + (int64_t)bg * p.T * p.topk + beg;
+    const uint32_t code0 = kStTimeoutBase + kKidFwd * 16;
+    if ((smem_u32(smem) & 1023u) != 0u) {   // the swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0) atomicCAS(p.status, 0u, code0 + 15);
+        return;
+    }
+    const int32_t* toks = p.tok + (int64_t)bg * p.T * p.topk + item.beg;
     const int nchunks = (count + p.tpc - 1) / p.tpc;
 
     uint8_t* k_tile = smem;
     uint8_t* v_tile = smem + kTile;
     uint8_t* q_st = smem + 2 * kTile;
-    uint64_t* bars = (uint64_t*)(q_st + kQStages * kTile);
+    // O staging: token t of a chunk at t * (G*D*4 + 16) bytes; the 16-byte pad
+    // per token spreads the rows of a warp over all banks.
+    uint8_t* o_stg = q_st + kQStages * kTile;
+    const uint32_t tok_bytes = (uint32_t)G * D * 4u;
+    const uint32_t tok_stride = tok_bytes + 16u;
+    uint64_t* bars = (uint64_t*)(o_stg + 128 * D * 4 + 2048);
     uint64_t* kv_full = bars;
     uint64_t* q_full = bars + 1;
     uint64_t* q_empty = q_full + kQStages;
@@ -85,7 +94,6 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint32_t* tmem_hold = (uint32_t*)(fin + 1);
     volatile uint32_t* abort_flag = tmem_hold + 1;
     const WaitCtx wc{p.status, abort_flag, MSA_WAIT_LIMIT_NS};
-    const uint32_t code0 = kStTimeoutBase + kKidFwd * 16;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -231,36 +239,54 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
     } else {
         // ---------------- O partials -> fp32 global accumulators ----------------
+        // TMEM -> padded staging in shared memory -> one bulk fp32 reduction of
+        // G*D floats per token (whole cache lines at L2 instead of 16-byte
+        // reductions from every thread).
+        // Each warp owns whole tokens (its 32 rows are 32/G tokens), so it
+        // stages and reduces them on its own, without waiting for the others.
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
+        const int t = r >> p.lgG, hh = r & (G - 1);
+        const int tpw = 32 >> p.lgG;                   // tokens per warp
+        const int my_tok = (warp & 3) * tpw + lane;    // token this lane reduces (lane < tpw)
+        const uint32_t stg = smem_u32(o_stg);
+        const uint32_t my_row = stg + (uint32_t)t * tok_stride + (uint32_t)hh * D * 4u;
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             const uint32_t use = (uint32_t)(c >> 1);
             const bool ok = mbar_wait(&o_full[buf], use & 1u, wc, code0 + 6);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const int jj = c * p.tpc + t;
-            const bool valid = jj < count;
-            const int i = valid ? toks[jj] : 0;
-            float* dst = p.oacc + (((int64_t)b * p.T + i) * p.Hq + h) * D;
+            // the previous chunk's bulk reductions must have read this warp's staging
+            if (lane < tpw) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
             const uint32_t ta = tmem_addr(tmem, lane_base, 256u + (uint32_t)buf * D);
 #pragma unroll
             for (int piece = 0; piece < D / 32; ++piece) {
                 uint32_t v[32];
                 tmem_ld32(ta + piece * 32, v);
                 tmem_ld_wait();
-                if (valid) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        red_add_v4(dst + piece * 32 + 4 * e, __uint_as_float(v[4 * e]),
-                                   __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
-                                   __uint_as_float(v[4 * e + 3]));
-                }
+                for (int e = 0; e < 8; ++e)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + (piece * 32 + 4 * e) * 4),
+                                 "r"(v[4 * e]), "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3])
+                                 : "memory");
             }
             tc_fence_before();
-            mbar_arrive(&o_empty[buf]);
+            mbar_arrive(&o_empty[buf]);     // the TMEM buffer is free once copied out
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int ntok = min(p.tpc, count - c * p.tpc);
+            if (lane < tpw && my_tok < ntok) {
+                const int i = toks[c * p.tpc + my_tok];
+                float* dst = p.oacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D;
+                asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+                             "r"(stg + (uint32_t)my_tok * tok_stride), "r"(tok_bytes)
+                             : "memory");
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
         }
+        if (lane < tpw) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
     __syncthreads();
@@ -465,15 +491,18 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     p.bound = fabsf(pr.scale) * kLog2e;
     p.q = qb;
     p.ptr = (const int32_t*)(w + L.ptr);
+    p.off = (const int32_t*)(w + L.cnt);
     p.tok = (const int32_t*)(w + L.tok);
     p.qn = qn; p.kmax = kmax; p.oacc = oacc; p.lacc = lacc;
     p.status = (uint32_t*)(w + L.status);
-    const size_t smem = 1024 + (size_t)(2 + kQStages) * 128 * D * 2 + 32 * 8;
+    p.RB = range_blocks(pr);
+    p.per_group = range_items_per_group(pr.nblk, p.RB);
+    const size_t smem = (size_t)(2 + kQStages) * 128 * D * 2 + 128 * D * 4 + 2048 + 32 * 8;
     if ((e = cudaFuncSetAttribute(fwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
     trace_begin(kTraceFwdMain, st);
-    fwd_main_kernel<D><<<(unsigned)(pr.nblk * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+    fwd_main_kernel<D><<<(unsigned)(p.per_group * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
     trace_end(kTraceFwdMain, st);
 
     const int64_t fth = (int64_t)pr.rows_q() * (D / 8);
