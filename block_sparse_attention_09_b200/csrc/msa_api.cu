@@ -156,8 +156,9 @@ int msa_proxy_select(const msa_dims* dims, const void* qp, const void* kp, int32
         return MSA_ERR_MISALIGNED;
     if ((rc = check_device()) != MSA_OK) return rc;
     CUtensorMap tq, tk;
+    // query tiles of 128 rows; key tiles of 256 rows (two key blocks per MMA)
     if (!make_tmap_bf16_4d(&tq, qp, p.dp, p.Hp, p.T, p.B, 64, 128) ||
-        !make_tmap_bf16_4d(&tk, kp, p.dp, p.Hp, p.T, p.B, 64, 128))
+        !make_tmap_bf16_4d(&tk, kp, p.dp, p.Hp, p.T, p.B, 64, 256))
         return MSA_ERR_DRIVER;
     cudaStream_t st = (cudaStream_t)stream;
     uint32_t* status = (uint32_t*)((uint8_t*)ws + L.status);

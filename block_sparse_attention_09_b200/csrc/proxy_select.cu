@@ -7,17 +7,30 @@
 //
 // One CTA owns one (batch, group, 128-query tile qb).  The proxy query tile
 // stays in shared memory; proxy key tiles n = 0 .. qb-1 stream in through a
-// 4-stage TMA ring; one thread issues tcgen05 MMAs (M=128 queries, N=128
-// keys, K=dp) into a double-buffered TMEM accumulator; four epilogue warps
-// (one TMEM lane = one query row each) reduce each 128-column tile to its
-// max and feed it into the row's selection heap in shared memory.  The
-// diagonal tile is needed only for the optional pooled-score output: the own
-// block is always selected, so selection only ranks blocks 0 .. qb-1, which
-// every query of the tile sees in full (no causal mask there).
+// TMA ring two key blocks at a time; one thread issues tcgen05 MMAs (M=128
+// queries, N=256 keys, K=dp: at N=128 an accumulation chain of dependent
+// MMAs runs at half rate) into two TMEM accumulators; eight epilogue warps (one TMEM lane = one
+// query row each; two warps per lane quarter, one per key block of the
+// 256-key MMA) reduce each 128-column block to its max and feed the row's
+// selection.  The diagonal tile is needed only for the optional
+// pooled-score output: the own block is always selected, so selection only
+// ranks blocks 0 .. qb-1, which every query of the tile sees in full.
 //
-// Selection order: higher pooled score first, equal scores to the lower
-// block id.  Tiles arrive in ascending n, so a later tile displaces the heap
-// root (the current worst) only with a strictly greater score.
+// Selection state per row (shared memory, [slot][row] so a warp touches 32
+// distinct banks): a 4-ary heap of the best topk-1 (score, id) pairs whose
+// root is the worst kept pair, and a small pending list.  At the end each
+// warp sorts its rows' kept ids with a bitonic network across its lanes.  Key tiles are
+// scanned nearest-first (descending block id): under causal locality the
+// best blocks tend to be the recent ones, so after the first few tiles a
+// new tile rarely beats the heap root.  A new tile has a lower id than every
+// kept pair, so it displaces the root when its score is greater or equal; a
+// tile beating the root (kept in a register) is appended to the pending
+// list, and the warp merges pending lists into the heaps only when one of
+// its rows fills its list.  Order: higher score first, equal scores to the
+// lower block id.
+//
+// CTAs run group by group, heaviest query tiles first, so the proxy keys of
+// one group stay in L2 while its tiles are processed.
 #include <math.h>
 
 #include "msa_device.cuh"
@@ -26,10 +39,9 @@
 namespace msa {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kThreads = 192;             // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr int kThreads = 320;             // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
 constexpr uint32_t kTileBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle slab)
-constexpr uint32_t kTmemCols = 256;        // two 128-column fp32 accumulators
+constexpr int kPend = 8;                   // pending candidates per row before a merge
 
 struct Params {
     int B, T, Hp, dp, nblk, topk;
@@ -44,22 +56,27 @@ MSA_DEV bool worse(float sa, int ia, float sb, int ib)
     return sa < sb || (sa == sb && ia > ib);
 }
 
-// Column r of the [slot][128] heap arrays: a binary heap whose root is the
-// worst kept candidate.
+// Column r of the [slot][128] heap arrays: a 4-ary heap whose root is the
+// worst kept candidate (children of x are 4x+1 .. 4x+4: half the depth of a
+// binary heap, and the four children are read in parallel).
 MSA_DEV void sift_down(float* hs, int* hi, int k1, int r, int x)
 {
     const float sx = hs[x * 128 + r];
     const int ix = hi[x * 128 + r];
     for (;;) {
-        const int l = 2 * x + 1;
-        if (l >= k1) break;
-        int w = l;
-        float sw = hs[l * 128 + r];
-        int iw = hi[l * 128 + r];
-        if (l + 1 < k1) {
-            const float s2 = hs[(l + 1) * 128 + r];
-            const int i2 = hi[(l + 1) * 128 + r];
-            if (worse(s2, i2, sw, iw)) { w = l + 1; sw = s2; iw = i2; }
+        const int c0 = 4 * x + 1;
+        if (c0 >= k1) break;
+        int w = c0;
+        float sw = hs[c0 * 128 + r];
+        int iw = hi[c0 * 128 + r];
+#pragma unroll
+        for (int d = 1; d < 4; ++d) {
+            const int c = c0 + d;
+            if (c < k1) {
+                const float sc = hs[c * 128 + r];
+                const int ic = hi[c * 128 + r];
+                if (worse(sc, ic, sw, iw)) { w = c; sw = sc; iw = ic; }
+            }
         }
         if (!worse(sw, iw, sx, ix)) break;
         hs[x * 128 + r] = sw;
@@ -70,39 +87,119 @@ MSA_DEV void sift_down(float* hs, int* hi, int k1, int r, int x)
     hi[x * 128 + r] = ix;
 }
 
+// Ascending sort of the 32*V ints a warp holds V per lane (element
+// V*lane + w in v[w]) by a bitonic network.
+template <int V>
+MSA_DEV void warp_sort(int (&v)[V])
+{
+    const int lane = (int)(threadIdx.x & 31u);
+#pragma unroll
+    for (int k = 2; k <= 32 * V; k <<= 1) {
+#pragma unroll
+        for (int s = k >> 1; s >= 1; s >>= 1) {
+            if (s < V) {   // partner in the same lane
+#pragma unroll
+                for (int w = 0; w < V; ++w) {
+                    const int wp = w ^ s;
+                    if (wp > w) {
+                        const bool up = ((V * lane + w) & k) == 0;
+                        const int a = v[w], b = v[wp];
+                        v[w] = up ? min(a, b) : max(a, b);
+                        v[wp] = up ? max(a, b) : min(a, b);
+                    }
+                }
+            } else {
+                const int ls = s / V;   // partner lane distance
+#pragma unroll
+                for (int w = 0; w < V; ++w) {
+                    const int j = V * lane + w;
+                    const int other = __shfl_xor_sync(0xffffffffu, v[w], ls);
+                    const bool up = (j & k) == 0, lower = (j & s) == 0;
+                    v[w] = (up == lower) ? min(v[w], other) : max(v[w], other);
+                }
+            }
+        }
+    }
+}
+
+// The warp's 32 rows (TMEM lane quarter q): ascending output of each row's
+// kept ids plus the own block, -1 padded; one row at a time, V ids per lane.
+template <int V>
+MSA_DEV void write_selection(const int* heap_i, int k1, int topk, int q, int qb, int T, int64_t row0,
+                             int32_t* idx, int32_t* nsel)
+{
+    const int lane = (int)(threadIdx.x & 31u);
+    for (int rr = 0; rr < 32; ++rr) {
+        const int row = q * 32 + rr;
+        int v[V];
+#pragma unroll
+        for (int w = 0; w < V; ++w) {
+            const int slot = V * lane + w;
+            v[w] = slot < k1 ? heap_i[slot * 128 + row] : 0x7fffffff;
+        }
+        warp_sort<V>(v);
+        const int i = qb * 128 + row;
+        if (i < T) {
+            int32_t* out = idx + (row0 + row) * topk;
+#pragma unroll
+            for (int w = 0; w < V; ++w) {
+                const int slot = V * lane + w;
+                if (slot < k1) out[slot] = v[w];
+                else if (slot == k1) out[slot] = qb;
+                else if (slot < topk) out[slot] = -1;
+            }
+            if (lane == 0) nsel[row0 + row] = k1 + 1;
+        }
+    }
+}
+
+// NSTAGE stages of 256 proxy keys (two key blocks) each; two TMEM
+// accumulators of 256 columns (all of TMEM: one CTA per SM).
+template <int NSTAGE>
 __global__ void __launch_bounds__(kThreads, 1)
 proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_kp,
                     Params p)
 {
+    constexpr int NACC = 2;
+    constexpr uint32_t kTmemCols = 512;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = p.B * p.Hp;
-    const int qb = p.nblk - 1 - (int)(blockIdx.x / BH);   // heaviest tiles first
-    const int bg = (int)(blockIdx.x % BH);
+    // group by group, heaviest (largest qb) tiles first within a group
+    const int bg = (int)(blockIdx.x / p.nblk);
+    const int qb = p.nblk - 1 - (int)(blockIdx.x % p.nblk);
     const int b = bg / p.Hp, g = bg % p.Hp;
     const int k1 = p.topk - 1;                             // slots besides the own block
     const bool dbg = p.pooled != nullptr;
     const bool take_all = qb + 1 <= p.topk;                // every eligible block kept
     const bool need_heap = !take_all && k1 > 0;
     const int ntiles = dbg ? qb + 1 : (need_heap ? qb : 0);
+    const int npairs = (ntiles + 1) / 2;
+    // pair k holds key blocks hi = ntiles-1-2k (nearest first) and lo = hi-1
+    // (lo = -1 past the first block: that half is zero-filled and ignored)
 
     // epilogue row of this thread (warps 2..5 own TMEM lane quarters 2,3,0,1)
     const int r = ((warp & 3) << 5) | lane;
     const int i = qb * 128 + r;
-    const bool row_ok = (warp >= 2) && (i < p.T);
+    const bool row_ok = (warp >= 2) && (warp < 6) && (i < p.T);   // the selection-owning warps
 
+    const int hk = k1 > 0 ? k1 : 0;
     uint8_t* qp_tile = smem;
     uint8_t* kp_tiles = smem + kTileBytes;
-    float* heap_s = (float*)(smem + kTileBytes * (1 + kStages));
-    int* heap_i = (int*)(heap_s + (size_t)(k1 > 0 ? k1 : 0) * 128);
-    uint64_t* bars = (uint64_t*)(heap_i + (size_t)(k1 > 0 ? k1 : 0) * 128);
-    uint64_t* full = bars;                 // [kStages] TMA -> MMA
-    uint64_t* empty = bars + kStages;      // [kStages] MMA -> TMA
-    uint64_t* acc_full = bars + 2 * kStages;   // [2] MMA -> epilogue
-    uint64_t* acc_empty = acc_full + 2;        // [2] epilogue -> MMA
-    uint64_t* qp_full = acc_empty + 2;
+    float* heap_s = (float*)(smem + kTileBytes * (1 + 2 * NSTAGE));
+    int* heap_i = (int*)(heap_s + (size_t)hk * 128);
+    float* pend_s = (float*)(heap_i + (size_t)hk * 128);
+    int* pend_i = (int*)(pend_s + kPend * 128);
+    float* xchg = (float*)(pend_i + kPend * 128);   // [2][128]: max of the farther block of a pair
+    uint64_t* bars = (uint64_t*)(xchg + 2 * 128);
+    uint64_t* full = bars;                     // [NSTAGE] TMA -> MMA
+    uint64_t* empty = bars + NSTAGE;           // [NSTAGE] MMA -> TMA
+    uint64_t* acc_full = bars + 2 * NSTAGE;    // [NACC] MMA -> epilogue
+    uint64_t* acc_empty = acc_full + NACC;     // [NACC] epilogue -> MMA
+    uint64_t* xchg_full = acc_empty + NACC;    // [2] far-block warps -> selection warps
+    uint64_t* xchg_empty = xchg_full + 2;      // [2] selection warps -> far-block warps
+    uint64_t* qp_full = xchg_empty + 2;
     uint64_t* fin = qp_full + 1;               // MMA teardown drain
     uint32_t* tmem_hold = (uint32_t*)(fin + 1);
     volatile uint32_t* abort_flag = tmem_hold + 1;
@@ -126,8 +223,9 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     }
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], 128); }
+        for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < NACC; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], 256); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&xchg_full[s], 128); mbar_init(&xchg_empty[s], 128); }
         mbar_init(qp_full, 1);
         mbar_init(fin, 1);
         *abort_flag = 0u;
@@ -140,45 +238,46 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     const uint32_t tmem = *tmem_hold;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer: one 256-key box per pair ----------------
         if (lane == 0) {
             tma_prefetch_desc(&tm_qp);
             tma_prefetch_desc(&tm_kp);
             mbar_arrive_expect_tx(qp_full, kTileBytes);
             tma_load_4d(qp_tile, &tm_qp, qp_full, 0, g, qb * 128, b);
-            int n = 0;
-            for (; n < ntiles; ++n) {
-                const int s = n % kStages;
-                const uint32_t use = (uint32_t)(n / kStages);
+            int k = 0;
+            for (; k < npairs; ++k) {
+                const int s = k % NSTAGE;
+                const uint32_t use = (uint32_t)(k / NSTAGE);
                 if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u, wc, code0 + 0)) break;
-                mbar_arrive_expect_tx(&full[s], kTileBytes);
-                tma_load_4d(kp_tiles + s * kTileBytes, &tm_kp, &full[s], 0, g, n * 128, b);
+                const int lo = ntiles - 2 - 2 * k;   // may be -1: rows before 0 read as zeros
+                mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
+                tma_load_4d(kp_tiles + s * 2 * kTileBytes, &tm_kp, &full[s], 0, g, lo * 128, b);
             }
             if (*abort_flag) {   // let copies still in flight land before the CTA exits
                 mbar_drain(qp_full, 0);
-                for (int m = (n > kStages ? n - kStages : 0); m < n; ++m)
-                    mbar_drain(&full[m % kStages], (uint32_t)(m / kStages) & 1u);
+                for (int m = (k > NSTAGE ? k - NSTAGE : 0); m < k; ++m)
+                    mbar_drain(&full[m % NSTAGE], (uint32_t)(m / NSTAGE) & 1u);
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+        // ---------------- MMA issuer: M = 128 queries, N = 256 keys ----------------
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, 128, false, false);
+            const uint32_t idesc = idesc_bf16(128, 256, false, false);
             const int ksteps = (p.dp + 15) / 16;
             const uint32_t a0 = smem_u32(qp_tile);
             bool ok = mbar_wait(qp_full, 0, wc, code0 + 1);
-            for (int n = 0; ok && n < ntiles; ++n) {
-                const int s = n % kStages;
-                const uint32_t use = (uint32_t)(n / kStages);
-                const int buf = n & 1;
-                const uint32_t ause = (uint32_t)(n >> 1);
+            for (int k = 0; ok && k < npairs; ++k) {
+                const int s = k % NSTAGE;
+                const uint32_t use = (uint32_t)(k / NSTAGE);
+                const int buf = k % NACC;
+                const uint32_t ause = (uint32_t)(k / NACC);
                 if (!mbar_wait(&full[s], use & 1u, wc, code0 + 2)) break;
                 if (ause > 0 && !mbar_wait(&acc_empty[buf], (ause - 1) & 1u, wc, code0 + 3)) break;
                 tc_fence_after();
-                const uint32_t b0 = smem_u32(kp_tiles + s * kTileBytes);
+                const uint32_t b0 = smem_u32(kp_tiles + s * 2 * kTileBytes);
                 for (int kk = 0; kk < ksteps; ++kk)
-                    umma_ss(tmem + buf * 128, desc_kmajor(a0, 128, kk * 16),
-                            desc_kmajor(b0, 128, kk * 16), idesc, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + buf * 256, desc_kmajor(a0, 128, kk * 16),
+                            desc_kmajor(b0, 256, kk * 16), idesc, kk > 0 ? 1u : 0u);
                 umma_commit(&empty[s]);
                 umma_commit(&acc_full[buf]);
             }
@@ -188,76 +287,119 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     } else {
         // ---------------- epilogue: pool + select ----------------
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        int cnt = 0;
-        for (int n = 0; n < ntiles; ++n) {
-            const int buf = n & 1;
-            const uint32_t use = (uint32_t)(n >> 1);
-            bool ok = mbar_wait(&acc_full[buf], use & 1u, wc, code0 + 4);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-            const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 128u);
-            const bool diag = (n == qb);
-            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t v[64];
-                tmem_ld32(ta + half * 64, v);
-                tmem_ld32(ta + half * 64 + 32, v + 32);
-                tmem_ld_wait();
-                if (diag) {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (half * 64 + c > r) v[c] = __float_as_uint(-INFINITY);
-                }
-#pragma unroll
-                for (int c = 0; c < 64; c += 8) {
-                    m0 = fmax3(m0, __uint_as_float(v[c + 0]), __uint_as_float(v[c + 1]));
-                    m1 = fmax3(m1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-                    m2 = fmax3(m2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
-                    m3 = fmax3(m3, __uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&acc_empty[buf]);
-            const float mx = fmaxf(fmax3(m0, m1, m2), m3);
-            if (dbg && row_ok) p.pooled[((int64_t)bg * p.T + i) * p.nblk + n] = mx;
-            if (need_heap && !diag) {
-                if (cnt < k1) {
-                    heap_s[cnt * 128 + r] = mx;
-                    heap_i[cnt * 128 + r] = n;
-                    if (++cnt == k1)
-                        for (int x = k1 / 2 - 1; x >= 0; --x) sift_down(heap_s, heap_i, k1, r, x);
-                } else if (mx > heap_s[r]) {
-                    heap_s[r] = mx;
-                    heap_i[r] = n;
+        int cnt = 0, npend = 0;
+        float tau = -INFINITY;   // score of the heap root once the heap is full
+        auto merge_pending = [&]() {
+            for (int e = 0; e < npend; ++e) {
+                const float sc = pend_s[e * 128 + r];
+                if (sc >= heap_s[r]) {   // lower id than every kept pair: ties go to it
+                    heap_s[r] = sc;
+                    heap_i[r] = pend_i[e * 128 + r];
                     sift_down(heap_s, heap_i, k1, r, 0);
                 }
             }
-        }
-        if (row_ok && !*abort_flag) {
-            int32_t* out = p.idx + ((int64_t)bg * p.T + i) * p.topk;
-            int c = 0;
-            if (take_all) {
-                for (int n = 0; n <= qb; ++n) out[c++] = n;
-            } else if (k1 == 0) {
-                out[c++] = qb;
-            } else {
-                // ascending block ids: insertion sort of the heap column
-                for (int a = 1; a < k1; ++a) {
-                    const int key = heap_i[a * 128 + r];
-                    int x = a - 1;
-                    while (x >= 0 && heap_i[x * 128 + r] > key) {
-                        heap_i[(x + 1) * 128 + r] = heap_i[x * 128 + r];
-                        --x;
-                    }
-                    heap_i[(x + 1) * 128 + r] = key;
-                }
-                for (int a = 0; a < k1; ++a) out[c++] = heap_i[a * 128 + r];
-                out[c++] = qb;
+            npend = 0;
+            tau = heap_s[r];
+        };
+        // max over one 128-key block (TMEM columns col0 .. col0+127); the own
+        // block is cut at the query (causal)
+        auto block_max = [&](uint32_t ta, bool diag) -> float {
+            uint32_t v[128];
+            tmem_ld32(ta, v);
+            tmem_ld32(ta + 32, v + 32);
+            tmem_ld32(ta + 64, v + 64);
+            tmem_ld32(ta + 96, v + 96);
+            tmem_ld_wait();
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c > r) v[c] = __float_as_uint(-INFINITY);
             }
-            p.nsel[(int64_t)bg * p.T + i] = c;
-            for (int s = c; s < p.topk; ++s) out[s] = -1;
-            if (dbg)
+            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; c += 8) {
+                m0 = fmax3(m0, __uint_as_float(v[c + 0]), __uint_as_float(v[c + 1]));
+                m1 = fmax3(m1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                m2 = fmax3(m2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
+                m3 = fmax3(m3, __uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
+            }
+            return fmaxf(fmax3(m0, m1, m2), m3);
+        };
+        auto consume = [&](int n, float mx) {
+            if (dbg && row_ok) p.pooled[((int64_t)bg * p.T + i) * p.nblk + n] = mx;
+            if (!need_heap || n == qb) return;
+            if (cnt < k1) {   // same count for every row of the tile: warp-uniform
+                heap_s[cnt * 128 + r] = mx;
+                heap_i[cnt * 128 + r] = n;
+                if (++cnt == k1) {
+                    for (int x = (k1 - 2) / 4; x >= 0; --x) sift_down(heap_s, heap_i, k1, r, x);
+                    tau = heap_s[r];
+                }
+            } else {
+                if (mx >= tau) {
+                    pend_s[npend * 128 + r] = mx;
+                    pend_i[npend * 128 + r] = n;
+                    ++npend;
+                }
+                if (__any_sync(0xffffffffu, npend == kPend)) merge_pending();
+            }
+        };
+        // warps 2-5 reduce the nearer block of each pair and own the selection
+        // state; warps 6-9 (same TMEM lane quarters) reduce the farther block
+        // and hand its max over through shared memory.
+        const bool sel_warp = warp < 6;
+        for (int k = 0; k < npairs; ++k) {
+            const int hi = ntiles - 1 - 2 * k, lo = hi - 1;
+            const int buf = k % NACC;
+            const uint32_t use = (uint32_t)(k / NACC);
+            bool ok = mbar_wait(&acc_full[buf], use & 1u, wc, code0 + 4);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 256u);
+            // columns 0..127: block lo, 128..255: block hi
+            if (sel_warp) {
+                const float mhi = block_max(ta + 128, hi == qb);
+                tc_fence_before();
+                mbar_arrive(&acc_empty[buf]);   // the accumulator is free for pair k + NACC
+                ok = mbar_wait(&xchg_full[k & 1], (uint32_t)(k >> 1) & 1u, wc, code0 + 5);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                const float mlo = xchg[(k & 1) * 128 + r];
+                mbar_arrive(&xchg_empty[k & 1]);
+                consume(hi, mhi);
+                if (lo >= 0) consume(lo, mlo);
+            } else {
+                const float mlo = lo >= 0 ? block_max(ta, false) : -INFINITY;
+                tc_fence_before();
+                mbar_arrive(&acc_empty[buf]);
+                if (k >= 2) {
+                    ok = mbar_wait(&xchg_empty[k & 1], (uint32_t)((k >> 1) - 1) & 1u, wc, code0 + 6);
+                    if (!__all_sync(0xffffffffu, ok)) break;
+                }
+                xchg[(k & 1) * 128 + r] = mlo;
+                mbar_arrive(&xchg_full[k & 1]);
+            }
+        }
+        if (sel_warp && need_heap && cnt == k1) merge_pending();
+        const bool go = __all_sync(0xffffffffu, !*abort_flag);
+        if (sel_warp && go) {
+            if (need_heap) {
+                const int64_t row0 = (int64_t)bg * p.T + qb * 128;
+                if (p.topk <= 64)
+                    write_selection<2>(heap_i, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+                else
+                    write_selection<4>(heap_i, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+            } else if (row_ok) {
+                int32_t* out = p.idx + ((int64_t)bg * p.T + i) * p.topk;
+                int c = 0;
+                if (take_all) {
+                    for (int n = 0; n <= qb; ++n) out[c++] = n;
+                } else {
+                    out[c++] = qb;
+                }
+                p.nsel[(int64_t)bg * p.T + i] = c;
+                for (int s = c; s < p.topk; ++s) out[s] = -1;
+            }
+            if (dbg && row_ok)
                 for (int n = qb + 1; n < p.nblk; ++n)
                     p.pooled[((int64_t)bg * p.T + i) * p.nblk + n] = -INFINITY;
         }
@@ -270,6 +412,27 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     }
 }
 
+template <int NSTAGE>
+cudaError_t launch_variant(const Problem& pr, const CUtensorMap& tm_qp, const CUtensorMap& tm_kp,
+                           const Params& p, size_t smem, cudaStream_t st)
+{
+    auto kern = proxy_select_kernel<NSTAGE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(pr.nblk * pr.B * pr.Hp);
+    trace_begin(kTraceProxy, st);
+    kern<<<grid, kThreads, smem, st>>>(tm_qp, tm_kp, p);
+    trace_end(kTraceProxy, st);
+    return cudaGetLastError();
+}
+
+size_t smem_bytes(int nstage, int topk)
+{
+    const size_t k1 = (size_t)(topk > 1 ? topk - 1 : 0);
+    return 1024 + (size_t)kTileBytes * (1 + 2 * nstage) + k1 * 128 * 8 + (size_t)kPend * 128 * 8 + 2 * 128 * 4 +
+           32 * 8 + 16;
+}
+
 }  // namespace
 
 cudaError_t launch_proxy_select(const Problem& pr, const CUtensorMap& tm_qp, const CUtensorMap& tm_kp,
@@ -277,16 +440,11 @@ cudaError_t launch_proxy_select(const Problem& pr, const CUtensorMap& tm_qp, con
                                 cudaStream_t st)
 {
     Params p{pr.B, pr.T, pr.Hp, pr.dp, pr.nblk, pr.topk, idx, nsel, pooled, status};
-    const size_t k1 = (size_t)(pr.topk - 1);
-    const size_t smem = 1024 + (size_t)kTileBytes * (1 + kStages) + k1 * 128 * 8 + 16 * 8 + 16;
-    cudaError_t e = cudaFuncSetAttribute(proxy_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)(pr.nblk * pr.B * pr.Hp);
-    trace_begin(kTraceProxy, st);
-    proxy_select_kernel<<<grid, kThreads, smem, st>>>(tm_qp, tm_kp, p);
-    trace_end(kTraceProxy, st);
-    return cudaGetLastError();
+    // All of TMEM per CTA: at least 120 KB of shared memory keeps one CTA per SM.
+    const size_t s4 = smem_bytes(4, pr.topk);
+    if (s4 <= 227 * 1024) return launch_variant<4>(pr, tm_qp, tm_kp, p, s4 < 120 * 1024 ? 120 * 1024 : s4, st);
+    const size_t s2 = smem_bytes(2, pr.topk);
+    return launch_variant<2>(pr, tm_qp, tm_kp, p, s2 < 120 * 1024 ? 120 * 1024 : s2, st);
 }
 
 }  // namespace msa

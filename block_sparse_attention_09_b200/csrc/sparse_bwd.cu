@@ -50,24 +50,36 @@ struct BwdParams {
 
 template <int D>
 struct BwdSmem {
-    static constexpr uint32_t kTile = 128u * D * 2u;
-    static constexpr uint32_t kK = 0, kV = kTile;
-    static constexpr uint32_t kStage0 = 2 * kTile;            // Q0, dO0, Q1, dO1
-    static constexpr uint32_t kDS = 6 * kTile;                 // dS tile (128 keys x 128 rows)
-    static constexpr uint32_t kMeta = kDS + 128 * 128 * 2;     // 2 x {L2[128], D[128], cmax[128]}
-    static constexpr uint32_t kMetaStage = 128 * 4 * 2 + 128;
-    static constexpr uint32_t kBars = kMeta + 2 * kMetaStage;
-    static constexpr uint32_t kNumBars = 12;
+    static constexpr int kStages = 4;                           // Q/dO ring
+    static constexpr uint32_t kKV = 128u * D * 2u;              // one K or V tile
+    static constexpr uint32_t kHalf = 64u * D * 2u;             // Q or dO of one 64-row chunk
+    static constexpr uint32_t kK = 0, kV = kKV;
+    static constexpr uint32_t kStage0 = 2 * kKV;                // stage s: Q at s*2*kHalf, dO after it
+    static constexpr uint32_t kDS = kStage0 + kStages * 2 * kHalf;   // 2 dS tiles (128 keys x 64 rows)
+    static constexpr uint32_t kDSTile = 128u * 64u * 2u;
+    static constexpr uint32_t kMeta = kDS + 2 * kDSTile;        // per stage {L2[64], D[64], cmax[64]}
+    static constexpr uint32_t kMetaStage = 64 * 4 * 2 + 64;
+    static constexpr uint32_t kBars = kMeta + kStages * kMetaStage;
+    static constexpr uint32_t kNumBars = 1 + 2 * kStages + 5 * 2 + 2;
     static constexpr uint32_t kTotal = kBars + kNumBars * 8 + 8;
+    static_assert(2 * 128 * (D * 4 + 16) <= kMeta - kStage0, "dK/dV staging must fit the stage and dS area");
 };
 
+// Work per item: the 64-row chunks (64/G tokens x G heads) of the item's
+// queries, software-pipelined over two TMEM buffer sets:
+//   MMA:      S^T(c), dP^T(c) -> buffer c&1      (issued two chunks ahead)
+//   softmax:  P^T, dS^T (bf16) into the same buffer, dS^T into smem tile c&1
+//   MMA:      dV += P^T dO, dK += dS^T Q, dQ^T = K^T dS^T (into dP^T's columns)
+//   epilogue: dQ^T -> this chunk's Q/dO stage (row-major) -> bulk fp32
+//             reduction per token; the stage is then free for chunk c+4.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 BwdParams p)
 {
     using SM = BwdSmem<D>;
-    constexpr uint32_t kTile = SM::kTile;
+    constexpr int kS = SM::kStages;
+    constexpr uint32_t kKV = SM::kKV, kHalf = SM::kHalf;
     constexpr int kSlabs = D / 64;
     extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -88,36 +100,38 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     uint8_t* k_tile = smem + SM::kK;
     uint8_t* v_tile = smem + SM::kV;
-    uint8_t* ds_tile = smem + SM::kDS;
     uint64_t* bars = (uint64_t*)(smem + SM::kBars);
-    uint64_t* kv_full = bars + 0;
-    uint64_t* st_full = bars + 1;    // [2]
-    uint64_t* st_empty = bars + 3;   // [2]
-    uint64_t* s_full = bars + 5;
-    uint64_t* p_full = bars + 6;
-    uint64_t* ds_empty = bars + 7;
-    uint64_t* dq_full = bars + 8;
-    uint64_t* dq_empty = bars + 9;
-    uint64_t* kv_done = bars + 10;
-    uint64_t* fin = bars + 11;
+    uint64_t* kv_full = bars;
+    uint64_t* st_full = bars + 1;           // [kS] producers -> MMA
+    uint64_t* st_empty = st_full + kS;      // [kS] dQ epilogue -> producers
+    uint64_t* s_full = st_empty + kS;       // [2] MMA -> softmax
+    uint64_t* p_full = s_full + 2;          // [2] softmax -> MMA
+    uint64_t* ds_empty = p_full + 2;        // [2] MMA (dQ^T read dS tile) -> softmax
+    uint64_t* dq_full = ds_empty + 2;       // [2] MMA -> dQ epilogue
+    uint64_t* dq_empty = dq_full + 2;       // [2] dQ epilogue (TMEM drained) -> MMA
+    uint64_t* kv_done = dq_empty + 2;
+    uint64_t* fin = kv_done + 1;
     uint32_t* tmem_hold = (uint32_t*)(bars + SM::kNumBars);
     volatile uint32_t* abort_flag = tmem_hold + 1;
     const WaitCtx wc{p.status, abort_flag, MSA_WAIT_LIMIT_NS};
 
-    auto q_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kTile; };
-    auto do_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kTile + kTile; };
+    auto q_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kHalf; };
+    auto do_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kHalf + kHalf; };
+    auto ds_tile = [&](int bb) { return smem + SM::kDS + (uint32_t)bb * SM::kDSTile; };
     auto meta_l2 = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage); };
-    auto meta_d = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage + 512); };
-    auto meta_cm = [&](int s) { return (int8_t*)(smem + SM::kMeta + s * SM::kMetaStage + 1024); };
+    auto meta_d = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage + 256); };
+    auto meta_cm = [&](int s) { return (int8_t*)(smem + SM::kMeta + s * SM::kMetaStage + 512); };
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        for (int s = 0; s < 2; ++s) { mbar_init(&st_full[s], 128); mbar_init(&st_empty[s], 1); }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
-        mbar_init(ds_empty, 1);
-        mbar_init(dq_full, 1);
-        mbar_init(dq_empty, 128);
+        for (int s = 0; s < kS; ++s) { mbar_init(&st_full[s], 128); mbar_init(&st_empty[s], 1); }
+        for (int bb = 0; bb < 2; ++bb) {
+            mbar_init(&s_full[bb], 1);
+            mbar_init(&p_full[bb], 128);
+            mbar_init(&ds_empty[bb], 1);
+            mbar_init(&dq_full[bb], 1);
+            mbar_init(&dq_empty[bb], 128);
+        }
         mbar_init(kv_done, 1);
         mbar_init(fin, 1);
         *abort_flag = 0u;
@@ -128,14 +142,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_hold;
-    // TMEM columns: S^T/P^T at 0, dP^T/dS^T/dQ at 128, dV at 256, dK at 256 + D.
-    const uint32_t tS = tmem, tdP = tmem + 128u, tdV = tmem + 256u, tdK = tmem + 256u + D;
+    // TMEM columns: buffer bb at bb*128: S^T/P^T [0,64), dP^T/dS^T/dQ^T [64,128);
+    // dV at 256, dK at 256 + D.
+    auto tS = [&](int bb) { return tmem + (uint32_t)bb * 128u; };
+    auto tdP = [&](int bb) { return tmem + (uint32_t)bb * 128u + 64u; };
+    const uint32_t tdV = tmem + 256u, tdK = tmem + 256u + D;
 
     if (warp == 0) {
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(kv_full, 2 * kTile);
+            mbar_arrive_expect_tx(kv_full, 2 * kKV);
             for (int s = 0; s < kSlabs; ++s) {
                 tma_load_4d(k_tile + s * 16384, &tm_k, kv_full, s * 64, g, n * 128, b);
                 tma_load_4d(v_tile + s * 16384, &tm_v, kv_full, s * 64, g, n * 128, b);
@@ -145,69 +162,68 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t idSS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
+            constexpr uint32_t idSS = idesc_bf16(128, 64, false, false);    // S^T, dP^T
             constexpr uint32_t idKV = idesc_bf16(128, D, false, true);      // dV, dK (A in TMEM)
-            constexpr uint32_t idQ = idesc_bf16(128, D, true, true);        // dQ (d = 64)
-            constexpr uint32_t idQT = idesc_bf16(128, 128, true, true);     // dQ^T (d = 128)
-            const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile), dsa = smem_u32(ds_tile);
-            bool ok = mbar_wait(kv_full, 0, wc, code0 + 0);
-            for (int c = 0; ok && c < nchunks; ++c) {
-                const int s = c & 1;
-                const uint32_t su = (uint32_t)(c >> 1);
-                if (!mbar_wait(&st_full[s], su & 1u, wc, code0 + 1)) break;
-                if (c > 0 && !mbar_wait(dq_empty, (uint32_t)(c - 1) & 1u, wc, code0 + 2)) break;
+            constexpr uint32_t idQT = idesc_bf16(128, 64, true, true);      // dQ^T (M = d, padded to 128)
+            const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile);
+            auto issue_pre = [&](int c) -> bool {   // S^T(c), dP^T(c)
+                const int s = c % kS, bb = c & 1;
+                if (!mbar_wait(&st_full[s], (uint32_t)(c / kS) & 1u, wc, code0 + 1)) return false;
+                if (c >= 2 && !mbar_wait(&dq_empty[bb], (uint32_t)((c - 2) >> 1) & 1u, wc, code0 + 2))
+                    return false;
                 tc_fence_after();
                 const uint32_t qa = smem_u32(q_stage(s)), oa = smem_u32(do_stage(s));
+                // S^T and dP^T are independent accumulation chains: interleaving
+                // their K-steps keeps more MMAs in flight than one chain at a time
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(tS, desc_kmajor(ka, 128, kk * 16), desc_kmajor(qa, 128, kk * 16), idSS,
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    umma_ss(tS(bb), desc_kmajor(ka, 128, kk * 16), desc_kmajor(qa, 64, kk * 16), idSS,
                             kk > 0 ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(tdP, desc_kmajor(va, 128, kk * 16), desc_kmajor(oa, 128, kk * 16), idSS,
+                    umma_ss(tdP(bb), desc_kmajor(va, 128, kk * 16), desc_kmajor(oa, 64, kk * 16), idSS,
                             kk > 0 ? 1u : 0u);
-                umma_commit(s_full);
-                if (!mbar_wait(p_full, (uint32_t)c & 1u, wc, code0 + 3)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tdV, tS + kk * 8, desc_mnmajor(oa, 128, kk * 16), idKV,
-                            (c > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tdK, tdP + kk * 8, desc_mnmajor(qa, 128, kk * 16), idKV,
-                            (c > 0 || kk > 0) ? 1u : 0u);
-                if constexpr (D == 128) {
-                    // dQ^T = K^T dS^T: one TMEM lane per head-dim index, so the
-                    // epilogue's reductions cover whole cache lines
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_ss(tdP, desc_mnmajor(ka, 128, kk * 16), desc_mnmajor(dsa, 128, kk * 16), idQT,
-                                kk > 0 ? 1u : 0u);
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_ss(tdP, desc_mnmajor(dsa, 128, kk * 16), desc_mnmajor(ka, 128, kk * 16), idQ,
-                                kk > 0 ? 1u : 0u);
                 }
-                // d = 128: the dQ epilogue stages through this chunk's Q/dO buffers
-                // and releases them itself once its bulk reductions have read them
-                if constexpr (D != 128) umma_commit(&st_empty[s]);
-                umma_commit(ds_empty);
-                umma_commit(dq_full);
+                umma_commit(&s_full[bb]);
+                return true;
+            };
+            bool ok = mbar_wait(kv_full, 0, wc, code0 + 0);
+            if (ok && nchunks > 0) ok = issue_pre(0);
+            if (ok && nchunks > 1) ok = issue_pre(1);
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int s = c % kS, bb = c & 1;
+                if (!mbar_wait(&p_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 3)) break;
+                tc_fence_after();
+                const uint32_t qa = smem_u32(q_stage(s)), oa = smem_u32(do_stage(s));
+                const uint32_t dsa = smem_u32(ds_tile(bb));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {   // K = 64 rows; dV and dK chains interleaved
+                    umma_ts(tdV, tS(bb) + kk * 8, desc_mnmajor(oa, 64, kk * 16), idKV,
+                            (c > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts(tdK, tdP(bb) + kk * 8, desc_mnmajor(qa, 64, kk * 16), idKV,
+                            (c > 0 || kk > 0) ? 1u : 0u);
+                }
+                // dQ^T = K^T dS^T over the 128 keys; with d = 64 the second half
+                // of the M = 128 tile reads the V tile and lands in TMEM lanes
+                // nobody reads.
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ss(tdP(bb), desc_mnmajor(ka, 128, kk * 16), desc_mnmajor(dsa, 128, kk * 16), idQT,
+                            kk > 0 ? 1u : 0u);
+                umma_commit(&ds_empty[bb]);
+                umma_commit(&dq_full[bb]);
+                if (c + 2 < nchunks) ok = issue_pre(c + 2);
             }
             umma_commit(kv_done);
             umma_commit(fin);
             mbar_drain(fin, 0);
         }
     } else if (warp < 6) {
-        // ---------------- gather Q, dO and per-row metadata ----------------
+        // ---------------- gather Q, dO (64 rows) and per-row metadata ----------------
         const int tid = threadIdx.x - 64;
-        constexpr int kPieces = 128 * D / 8;
+        constexpr int kPieces = 64 * D / 8;
         constexpr int kRowPieces = D / 8;
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
-            const uint32_t su = (uint32_t)(c >> 1);
+            const int s = c % kS;
+            const uint32_t su = (uint32_t)(c / kS);
             if (su > 0 && !mbar_wait(&st_empty[s], (su - 1) & 1u, wc, code0 + 4)) break;
             const uint32_t qs = smem_u32(q_stage(s)), os = smem_u32(do_stage(s));
 #pragma unroll 4
@@ -219,11 +235,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const bool valid = jj < count;
                 const int i = valid ? toks[jj] : 0;
                 const int64_t off = (((int64_t)b * p.T + i) * p.Hq + g * G + hh) * D + ch * 8;
-                const uint32_t dst = sw128_offset(row, ch & 7, ch >> 3, 128);
+                const uint32_t dst = sw128_offset(row, ch & 7, ch >> 3, 64);
                 cp_async_16(qs + dst, p.q + off, valid ? 16u : 0u);
                 cp_async_16(os + dst, p.dout + off, valid ? 16u : 0u);
             }
-            {
+            if (tid < 64) {
                 const int row = tid;
                 const int t = row >> p.lgG, hh = row & (G - 1), h = g * G + hh;
                 const int jj = c * p.tpc + t;
@@ -244,19 +260,19 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // ---------------- P^T, dS^T (one TMEM lane = one key) ----------------
         const int jl = ((warp & 3) << 5) | lane;   // key within the block
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        const uint32_t aS = tmem_addr(tS, lane_base, 0), aP = tmem_addr(tdP, lane_base, 0);
-        const uint32_t dsa = smem_u32(ds_tile);
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
-            bool ok = mbar_wait(s_full, (uint32_t)c & 1u, wc, code0 + 5);
-            if (ok && c > 0) ok = mbar_wait(ds_empty, (uint32_t)(c - 1) & 1u, wc, code0 + 6);
+            const int s = c % kS, bb = c & 1;
+            bool ok = mbar_wait(&s_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 5);
+            if (ok && c >= 2) ok = mbar_wait(&ds_empty[bb], (uint32_t)((c - 2) >> 1) & 1u, wc, code0 + 6);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const float* L2 = meta_l2(s);
             const float* Dv = meta_d(s);
             const int8_t* cm = meta_cm(s);
+            const uint32_t aS = tmem_addr(tS(bb), lane_base, 0), aP = tmem_addr(tdP(bb), lane_base, 0);
+            const uint32_t dsa = smem_u32(ds_tile(bb));
 #pragma unroll
-            for (int piece = 0; piece < 4; ++piece) {
+            for (int piece = 0; piece < 2; ++piece) {
                 uint32_t sv[32], dv[32], pk[16], dk[16];
                 tmem_ld32(aS + piece * 32, sv);
                 tmem_ld32(aP + piece * 32, dv);
@@ -278,10 +294,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tmem_st16(aS + piece * 16, pk);   // P^T over S^T columns already read
                 tmem_st16(aP + piece * 16, dk);   // dS^T over dP^T columns already read
                 // dS^T row jl (rows piece*32 .. +31) into the MN-major dS tile
-                const uint32_t slab = (uint32_t)piece >> 1, cb = ((uint32_t)piece & 1u) * 4u;
 #pragma unroll
                 for (int qd = 0; qd < 4; ++qd) {
-                    const uint32_t addr = dsa + sw128_offset((uint32_t)jl, cb + qd, slab, 128);
+                    const uint32_t addr = dsa + sw128_offset((uint32_t)jl, (uint32_t)(piece * 4 + qd), 0, 128);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * qd]),
                                  "r"(dk[4 * qd + 1]), "r"(dk[4 * qd + 2]), "r"(dk[4 * qd + 3])
                                  : "memory");
@@ -290,82 +305,55 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tmem_st_wait();
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[bb]);
         }
     } else {
         // ---------------- dQ partials out; dK, dV partials at the end ----------------
-        const int r = ((warp & 3) << 5) | lane;    // TMEM lane of this thread
+        const int r = ((warp & 3) << 5) | lane;    // TMEM lane = head-dim index of dQ^T
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        const int tid = threadIdx.x - 320;
+        const uint32_t tok_bytes = (uint32_t)G * D * 4u;
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
-            ok = mbar_wait(dq_full, (uint32_t)c & 1u, wc, code0 + 7);
+            const int s = c % kS, bb = c & 1;
+            ok = mbar_wait(&dq_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 7);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t ta = tmem_addr(tdP, lane_base, 0);
-            const int ntok = min(p.tpc, count - c * p.tpc);
-            if constexpr (D == 128) {
-                // lane r holds dQ^T[r][row] for the chunk's 128 rows.  Stage them
-                // row-major ([row][d], the global order of a token's G heads) in
-                // this chunk's Q/dO buffers -- every store of a row is 32
-                // consecutive floats, no bank conflicts -- then reduce each token's
-                // G*D floats with one bulk operation.
-                const int s = c & 1;
-                const uint32_t stg = smem_u32(q_stage(s));
-#pragma unroll
-                for (int piece = 0; piece < 4; ++piece) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + piece * 32, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + ((piece * 32 + e) * D + r) * 4),
-                                     "r"(v[e])
-                                     : "memory");
-                }
-                tc_fence_before();
-                mbar_arrive(dq_empty);
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                const int tid = threadIdx.x - 320;
-                const uint32_t tok_bytes = (uint32_t)G * D * 4u;
-                for (int t = tid; t < ntok; t += 128) {
-                    const int i = toks[c * p.tpc + t];
-                    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                                     p.dqacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D),
-                                 "r"(stg + (uint32_t)t * tok_bytes), "r"(tok_bytes)
-                                 : "memory");
-                }
-                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                named_bar_sync(1, 128);
-                if (tid == 0) mbar_arrive(&st_empty[s]);
-                continue;
-            } else {
-                const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
-                const bool valid = t < ntok;
-                const int i = valid ? toks[c * p.tpc + t] : 0;
-                float* dst = p.dqacc + (((int64_t)b * p.T + i) * p.Hq + h) * D;
-#pragma unroll
-                for (int piece = 0; piece < D / 32; ++piece) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + piece * 32, v);
-                    tmem_ld_wait();
-                    if (valid) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            red_add_v4(dst + piece * 32 + 4 * e, __uint_as_float(v[4 * e]),
-                                       __uint_as_float(v[4 * e + 1]), __uint_as_float(v[4 * e + 2]),
-                                       __uint_as_float(v[4 * e + 3]));
-                    }
-                }
-            }
+            // dQ^T[r][row] for the chunk's 64 rows -> row-major staging in this
+            // chunk's Q/dO stage (32 consecutive floats per warp store)
+            const uint32_t stg = smem_u32(q_stage(s));
+            uint32_t v[64];
+            tmem_ld32(tmem_addr(tdP(bb), lane_base, 0), v);
+            tmem_ld32(tmem_addr(tdP(bb), lane_base, 32), v + 32);
+            tmem_ld_wait();
             tc_fence_before();
-            mbar_arrive(dq_empty);
+            mbar_arrive(&dq_empty[bb]);     // TMEM columns free for chunk c+2
+            if (r < D) {
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + ((uint32_t)e * D + (uint32_t)r) * 4u),
+                                 "r"(v[e])
+                                 : "memory");
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            const int ntok = min(p.tpc, count - c * p.tpc);
+            for (int t = tid; t < ntok; t += 128) {
+                const int i = toks[c * p.tpc + t];
+                asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                                 p.dqacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D),
+                             "r"(stg + (uint32_t)t * tok_bytes), "r"(tok_bytes)
+                             : "memory");
+            }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            named_bar_sync(1, 128);
+            if (tid == 0) mbar_arrive(&st_empty[s]);
         }
         if (ok) ok = mbar_wait(kv_done, 0, wc, code0 + 8);
         if (__all_sync(0xffffffffu, ok)) {
             // This item's dK, dV partials (lane = key) -> padded staging in the
-            // now idle Q/dO stages -> one bulk fp32 reduction per key row.
+            // now idle stage and dS area -> one bulk fp32 reduction per key row.
             tc_fence_after();
             const uint32_t row_stride = D * 4u + 16u;
             const uint32_t stg = smem_u32(smem + SM::kStage0);
@@ -376,13 +364,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const uint32_t row = stg + (uint32_t)which * 128u * row_stride + (uint32_t)r * row_stride;
 #pragma unroll
                 for (int piece = 0; piece < D / 32; ++piece) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + piece * 32, v);
+                    uint32_t w[32];
+                    tmem_ld32(ta + piece * 32, w);
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (piece * 32 + 4 * e) * 4),
-                                     "r"(v[4 * e]), "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3])
+                                     "r"(w[4 * e]), "r"(w[4 * e + 1]), "r"(w[4 * e + 2]), "r"(w[4 * e + 3])
                                      : "memory");
                 }
             }
@@ -483,7 +471,7 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     BwdParams p;
     p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
     p.lgG = 31 - __builtin_clz((unsigned)pr.G);
-    p.tpc = 128 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;
+    p.tpc = 64 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;   // 64-row chunks
     p.c1 = pr.scale * kLog2e;
     p.scale = pr.scale;
     p.q = (const __nv_bfloat16*)q;

@@ -133,6 +133,8 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idPV = idesc_bf16(128, D, false, true);
             const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile), qa = smem_u32(q_st);
+            // S(c+2) reuses the TMEM columns where P(c) lives, so it is issued
+            // only after every K-step of PV(c) (MMAs of one thread run in order).
             auto issue_s = [&](int c) -> bool {
                 const int s = c % kQStages;
                 const uint32_t use = (uint32_t)(c / kQStages);
@@ -202,17 +204,27 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
         const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
         const float kmx = p.kmax[bg];
+        const float* qn_row = p.qn + ((int64_t)b * p.Hq + h) * p.T;
+        // this row's token and |q| are loaded one and two chunks ahead, so the
+        // dependent global loads overlap the previous chunk's work
+        auto tok_of = [&](int cc) { const int jj = cc * p.tpc + t; return jj < count ? toks[jj] : -1; };
+        int tok_cur = tok_of(0), tok_nxt = nchunks > 1 ? tok_of(1) : -1;
+        float qn_cur = tok_cur >= 0 ? qn_row[tok_cur] : 0.f;
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             const uint32_t use = (uint32_t)(c >> 1);
+            const int tok_nn = c + 2 < nchunks ? tok_of(c + 2) : -1;
+            const float qn_nxt = tok_nxt >= 0 ? qn_row[tok_nxt] : 0.f;
             const bool ok = mbar_wait(&s_full[buf], use & 1u, wc, code0 + 5);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const int jj = c * p.tpc + t;
-            const bool valid = jj < count;
-            const int i = valid ? toks[jj] : 0;
+            const bool valid = tok_cur >= 0;
+            const int i = valid ? tok_cur : 0;
             const int cmax = valid ? (((i >> 7) == n) ? (i & 127) : 127) : -1;
-            const float mh = valid ? p.bound * p.qn[((int64_t)b * p.Hq + h) * p.T + i] * kmx : 0.f;
+            const float mh = valid ? p.bound * qn_cur * kmx : 0.f;
+            tok_cur = tok_nxt;
+            tok_nxt = tok_nn;
+            qn_cur = qn_nxt;
             const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 128u);
             float l = 0.f;
 #pragma unroll
@@ -251,6 +263,7 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int my_tok = (warp & 3) * tpw + lane;    // token this lane reduces (lane < tpw)
         const uint32_t stg = smem_u32(o_stg);
         const uint32_t my_row = stg + (uint32_t)t * tok_stride + (uint32_t)hh * D * 4u;
+        int my_tok_id = (lane < tpw && my_tok < count) ? toks[my_tok] : 0;
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             const uint32_t use = (uint32_t)(c >> 1);
@@ -277,8 +290,10 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             fence_proxy_async_smem();
             __syncwarp();
             const int ntok = min(p.tpc, count - c * p.tpc);
+            const int i = my_tok_id;
+            my_tok_id = (lane < tpw && c + 1 < nchunks && (c + 1) * p.tpc + my_tok < count)
+                            ? toks[(c + 1) * p.tpc + my_tok] : 0;   // next chunk's, loaded early
             if (lane < tpw && my_tok < ntok) {
-                const int i = toks[c * p.tpc + my_tok];
                 float* dst = p.oacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D;
                 asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
                              "r"(stg + (uint32_t)my_tok * tok_stride), "r"(tok_bytes)
