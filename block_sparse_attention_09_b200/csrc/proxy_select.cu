@@ -41,7 +41,7 @@ namespace {
 
 constexpr int kThreads = 320;             // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
 constexpr uint32_t kTileBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle slab)
-constexpr int kPend = 8;                   // pending candidates per row before a merge
+constexpr int kPend = 10;                  // pending slots per row (merge once one row holds 8)
 
 struct Params {
     int B, T, Hp, dp, nblk, topk;
@@ -51,40 +51,38 @@ struct Params {
     uint32_t* status;
 };
 
-MSA_DEV bool worse(float sa, int ia, float sb, int ib)
+// A candidate is (score bits, block id) in one 64-bit word.
+MSA_DEV uint2 cand(float s, int n) { return make_uint2(__float_as_uint(s), (uint32_t)n); }
+
+MSA_DEV bool worse(uint2 a, uint2 b)
 {
-    return sa < sb || (sa == sb && ia > ib);
+    const float sa = __uint_as_float(a.x), sb = __uint_as_float(b.x);
+    return sa < sb || (sa == sb && (int)a.y > (int)b.y);
 }
 
-// Column r of the [slot][128] heap arrays: a 4-ary heap whose root is the
+// Column r of the [slot][128] heap array: a 4-ary heap whose root is the
 // worst kept candidate (children of x are 4x+1 .. 4x+4: half the depth of a
-// binary heap, and the four children are read in parallel).
-MSA_DEV void sift_down(float* hs, int* hi, int k1, int r, int x)
+// binary heap; the four children are loaded together, indices past the end
+// repeating the last child).
+MSA_DEV void sift_down(uint2* h, int k1, int r, int x)
 {
-    const float sx = hs[x * 128 + r];
-    const int ix = hi[x * 128 + r];
+    const uint2 ex = h[x * 128 + r];
+    const int last = k1 - 1;
     for (;;) {
         const int c0 = 4 * x + 1;
-        if (c0 >= k1) break;
+        if (c0 > last) break;
+        const int c1 = min(c0 + 1, last), c2 = min(c0 + 2, last), c3 = min(c0 + 3, last);
+        const uint2 e0 = h[c0 * 128 + r], e1 = h[c1 * 128 + r], e2 = h[c2 * 128 + r], e3 = h[c3 * 128 + r];
         int w = c0;
-        float sw = hs[c0 * 128 + r];
-        int iw = hi[c0 * 128 + r];
-#pragma unroll
-        for (int d = 1; d < 4; ++d) {
-            const int c = c0 + d;
-            if (c < k1) {
-                const float sc = hs[c * 128 + r];
-                const int ic = hi[c * 128 + r];
-                if (worse(sc, ic, sw, iw)) { w = c; sw = sc; iw = ic; }
-            }
-        }
-        if (!worse(sw, iw, sx, ix)) break;
-        hs[x * 128 + r] = sw;
-        hi[x * 128 + r] = iw;
+        uint2 ew = e0;
+        if (worse(e1, ew)) { w = c1; ew = e1; }
+        if (worse(e2, ew)) { w = c2; ew = e2; }
+        if (worse(e3, ew)) { w = c3; ew = e3; }
+        if (!worse(ew, ex)) break;
+        h[x * 128 + r] = ew;
         x = w;
     }
-    hs[x * 128 + r] = sx;
-    hi[x * 128 + r] = ix;
+    h[x * 128 + r] = ex;
 }
 
 // Ascending sort of the 32*V ints a warp holds V per lane (element
@@ -125,7 +123,7 @@ MSA_DEV void warp_sort(int (&v)[V])
 // The warp's 32 rows (TMEM lane quarter q): ascending output of each row's
 // kept ids plus the own block, -1 padded; one row at a time, V ids per lane.
 template <int V>
-MSA_DEV void write_selection(const int* heap_i, int k1, int topk, int q, int qb, int T, int64_t row0,
+MSA_DEV void write_selection(const uint2* heap, int k1, int topk, int q, int qb, int T, int64_t row0,
                              int32_t* idx, int32_t* nsel)
 {
     const int lane = (int)(threadIdx.x & 31u);
@@ -135,7 +133,7 @@ MSA_DEV void write_selection(const int* heap_i, int k1, int topk, int q, int qb,
 #pragma unroll
         for (int w = 0; w < V; ++w) {
             const int slot = V * lane + w;
-            v[w] = slot < k1 ? heap_i[slot * 128 + row] : 0x7fffffff;
+            v[w] = slot < k1 ? (int)heap[slot * 128 + row].y : 0x7fffffff;
         }
         warp_sort<V>(v);
         const int i = qb * 128 + row;
@@ -187,11 +185,9 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     const int hk = k1 > 0 ? k1 : 0;
     uint8_t* qp_tile = smem;
     uint8_t* kp_tiles = smem + kTileBytes;
-    float* heap_s = (float*)(smem + kTileBytes * (1 + 2 * NSTAGE));
-    int* heap_i = (int*)(heap_s + (size_t)hk * 128);
-    float* pend_s = (float*)(heap_i + (size_t)hk * 128);
-    int* pend_i = (int*)(pend_s + kPend * 128);
-    float* xchg = (float*)(pend_i + kPend * 128);   // [2][128]: max of the farther block of a pair
+    uint2* heap = (uint2*)(smem + kTileBytes * (1 + 2 * NSTAGE));   // [topk-1][128]
+    uint2* pend = heap + (size_t)hk * 128;                             // [kPend][128]
+    float* xchg = (float*)(pend + kPend * 128);   // [2][128]: max of the farther block of a pair
     uint64_t* bars = (uint64_t*)(xchg + 2 * 128);
     uint64_t* full = bars;                     // [NSTAGE] TMA -> MMA
     uint64_t* empty = bars + NSTAGE;           // [NSTAGE] MMA -> TMA
@@ -291,15 +287,14 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
         float tau = -INFINITY;   // score of the heap root once the heap is full
         auto merge_pending = [&]() {
             for (int e = 0; e < npend; ++e) {
-                const float sc = pend_s[e * 128 + r];
-                if (sc >= heap_s[r]) {   // lower id than every kept pair: ties go to it
-                    heap_s[r] = sc;
-                    heap_i[r] = pend_i[e * 128 + r];
-                    sift_down(heap_s, heap_i, k1, r, 0);
+                const uint2 c = pend[e * 128 + r];
+                if (__uint_as_float(c.x) >= __uint_as_float(heap[r].x)) {   // lower id than every kept
+                    heap[r] = c;                                            // pair: ties go to it
+                    sift_down(heap, k1, r, 0);
                 }
             }
             npend = 0;
-            tau = heap_s[r];
+            tau = __uint_as_float(heap[r].x);
         };
         // max over one 128-key block (TMEM columns col0 .. col0+127); the own
         // block is cut at the query (causal)
@@ -329,19 +324,14 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
             if (dbg && row_ok) p.pooled[((int64_t)bg * p.T + i) * p.nblk + n] = mx;
             if (!need_heap || n == qb) return;
             if (cnt < k1) {   // same count for every row of the tile: warp-uniform
-                heap_s[cnt * 128 + r] = mx;
-                heap_i[cnt * 128 + r] = n;
+                heap[cnt * 128 + r] = cand(mx, n);
                 if (++cnt == k1) {
-                    for (int x = (k1 - 2) / 4; x >= 0; --x) sift_down(heap_s, heap_i, k1, r, x);
-                    tau = heap_s[r];
+                    for (int x = (k1 - 2) / 4; x >= 0; --x) sift_down(heap, k1, r, x);
+                    tau = __uint_as_float(heap[r].x);
                 }
-            } else {
-                if (mx >= tau) {
-                    pend_s[npend * 128 + r] = mx;
-                    pend_i[npend * 128 + r] = n;
-                    ++npend;
-                }
-                if (__any_sync(0xffffffffu, npend == kPend)) merge_pending();
+            } else if (mx >= tau) {
+                pend[npend * 128 + r] = cand(mx, n);
+                ++npend;
             }
         };
         // warps 2-5 reduce the nearer block of each pair and own the selection
@@ -367,6 +357,9 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
                 mbar_arrive(&xchg_empty[k & 1]);
                 consume(hi, mhi);
                 if (lo >= 0) consume(lo, mlo);
+                // one vote per pair: at most two appends per pair, so a list
+                // holding 8 still has room for the next pair
+                if (need_heap && cnt == k1 && __any_sync(0xffffffffu, npend >= kPend - 2)) merge_pending();
             } else {
                 const float mlo = lo >= 0 ? block_max(ta, false) : -INFINITY;
                 tc_fence_before();
@@ -385,9 +378,9 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
             if (need_heap) {
                 const int64_t row0 = (int64_t)bg * p.T + qb * 128;
                 if (p.topk <= 64)
-                    write_selection<2>(heap_i, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+                    write_selection<2>(heap, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
                 else
-                    write_selection<4>(heap_i, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+                    write_selection<4>(heap, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
             } else if (row_ok) {
                 int32_t* out = p.idx + ((int64_t)bg * p.T + i) * p.topk;
                 int c = 0;
