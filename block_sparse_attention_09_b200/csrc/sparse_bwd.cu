@@ -316,8 +316,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kS, bb = c & 1;
-            ok = mbar_wait(&dq_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 7);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ok = bar_and_sync(1, 128, mbar_wait(&dq_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 7));
+            if (!ok) break;   // all four warps leave together: none is left at a barrier below
             tc_fence_after();
             // dQ^T[r][row] for the chunk's 64 rows -> row-major staging in this
             // chunk's Q/dO stage (32 consecutive floats per warp store)

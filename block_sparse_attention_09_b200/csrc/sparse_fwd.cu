@@ -9,7 +9,8 @@
 // KV-stationary design.  One CTA owns one KV block n of one group: its K and
 // V tiles (128 keys) are loaded once by TMA; the queries that selected the
 // block are gathered from the inverse index in chunks of 128 rows (128/G
-// tokens x the G query heads of the group) with cp.async into a 3-stage ring.
+// tokens x the G query heads of the group, head-major: row = hh * 128/G + t)
+// with cp.async into a 3-stage ring.
 // Per chunk:  S = Q K^T (tcgen05, TMEM) -> P = exp(S*scale - bound) written
 // back to TMEM as bf16 -> O_part = P V (tcgen05 with A from TMEM) -> fp32
 // reductions of O_part and of the row sums into global accumulators.
@@ -184,7 +185,7 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int it = 0; it < kPieces / 128; ++it) {
                 const int piece = it * 128 + tid;
                 const int row = piece / kRowPieces, ch = piece % kRowPieces;
-                const int t = row >> p.lgG, hh = row & (G - 1);
+                const int t = row & (p.tpc - 1), hh = row >> (7 - p.lgG);
                 const int jj = c * p.tpc + t;
                 const bool valid = jj < count;
                 const int i = valid ? toks[jj] : 0;
@@ -202,7 +203,7 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // ---------------- softmax: P = exp2(S*c1 - bound) ----------------
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        const int t = r >> p.lgG, hh = r & (G - 1), h = g * G + hh;
+        const int t = r & (p.tpc - 1), hh = r >> (7 - p.lgG), h = g * G + hh;
         const float kmx = p.kmax[bg];
         const float* qn_row = p.qn + ((int64_t)b * p.Hq + h) * p.T;
         // this row's token and |q| are loaded one and two chunks ahead, so the
@@ -253,26 +254,25 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // ---------------- O partials -> fp32 global accumulators ----------------
         // TMEM -> padded staging in shared memory -> one bulk fp32 reduction of
         // G*D floats per token (whole cache lines at L2 instead of 16-byte
-        // reductions from every thread).
-        // Each warp owns whole tokens (its 32 rows are 32/G tokens), so it
-        // stages and reduces them on its own, without waiting for the others.
+        // reductions from every thread).  Rows are head-major, so the eight
+        // lanes of one 16-byte store phase hold eight different tokens and the
+        // per-token pad puts them on eight different bank groups.
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        const int t = r >> p.lgG, hh = r & (G - 1);
-        const int tpw = 32 >> p.lgG;                   // tokens per warp
-        const int my_tok = (warp & 3) * tpw + lane;    // token this lane reduces (lane < tpw)
+        const int t = r & (p.tpc - 1), hh = r >> (7 - p.lgG);
+        const int tid = threadIdx.x - 320;             // token this thread reduces
         const uint32_t stg = smem_u32(o_stg);
         const uint32_t my_row = stg + (uint32_t)t * tok_stride + (uint32_t)hh * D * 4u;
-        int my_tok_id = (lane < tpw && my_tok < count) ? toks[my_tok] : 0;
+        int my_tok_id = tid < min(p.tpc, count) ? toks[tid] : 0;
+        bool issued = false;
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             const uint32_t use = (uint32_t)(c >> 1);
             const bool ok = mbar_wait(&o_full[buf], use & 1u, wc, code0 + 6);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            // the previous chunk's bulk reductions must have read the staging
+            if (issued) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            if (!bar_and_sync(2, 128, ok)) break;   // all four warps go on, or none
             tc_fence_after();
-            // the previous chunk's bulk reductions must have read this warp's staging
-            if (lane < tpw) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-            __syncwarp();
             const uint32_t ta = tmem_addr(tmem, lane_base, 256u + (uint32_t)buf * D);
 #pragma unroll
             for (int piece = 0; piece < D / 32; ++piece) {
@@ -288,20 +288,21 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&o_empty[buf]);     // the TMEM buffer is free once copied out
             fence_proxy_async_smem();
-            __syncwarp();
+            named_bar_sync(2, 128);
             const int ntok = min(p.tpc, count - c * p.tpc);
             const int i = my_tok_id;
-            my_tok_id = (lane < tpw && c + 1 < nchunks && (c + 1) * p.tpc + my_tok < count)
-                            ? toks[(c + 1) * p.tpc + my_tok] : 0;   // next chunk's, loaded early
-            if (lane < tpw && my_tok < ntok) {
+            my_tok_id = (c + 1 < nchunks && tid < p.tpc && (c + 1) * p.tpc + tid < count)
+                            ? toks[(c + 1) * p.tpc + tid] : 0;   // next chunk's, loaded early
+            issued = tid < ntok;
+            if (issued) {
                 float* dst = p.oacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D;
                 asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
-                             "r"(stg + (uint32_t)my_tok * tok_stride), "r"(tok_bytes)
+                             "r"(stg + (uint32_t)tid * tok_stride), "r"(tok_bytes)
                              : "memory");
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             }
         }
-        if (lane < tpw) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        if (issued) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
     __syncthreads();
