@@ -9,16 +9,22 @@
 //   dV = P^T dO,  dK = dS^T Q,  dQ = dS K.
 //
 // KV-stationary: one CTA owns KV block n of one group, keeps K and V in
-// shared memory and dK, dV as fp32 accumulators in TMEM for the whole
-// bucket, so dK/dV need no atomics.  Chunks of 128 query rows (128/G tokens
-// x G heads) are gathered with cp.async (Q, dO, plus each row's L, D and
-// causal limit) into a 2-stage ring.  Per chunk, in the transposed
-// orientation so that one TMEM lane is one key:
-//   S^T = K Q^T, dP^T = V dO^T                 (tcgen05, A and B in smem)
-//   P^T, dS^T  -> TMEM (bf16) and dS^T -> smem  (softmax warps, lane = key)
-//   dV += P^T dO, dK += dS^T Q                  (tcgen05, A from TMEM)
-//   dQ_part = dS K                              (tcgen05, A = dS from smem)
-//   dQ_part -> fp32 reductions into a global accumulator (lane = query row).
+// shared memory and dK, dV as fp32 accumulators in TMEM for the whole work
+// item, so dK/dV need no atomics.  The queries that selected the block are
+// gathered with cp.async in chunks of 128 rows (128/G tokens x G heads) into
+// a 2-stage ring.  Per chunk, in the transposed orientation so that one TMEM
+// lane is one key, and with every MMA 128 wide (an M=128 tcgen05 MMA costs
+// about the same per instruction at N=64 as at N=128):
+//   S^T = K Q^T -> TMEM [0,128),  dP^T = V dO^T -> TMEM [128,256)
+//   softmax warps: P^T (bf16) over the S^T columns already read, and
+//                  dS^T = P^T (dP^T scale - D scale) (bf16) into a shared-memory tile
+//   dV += P^T dO (A from TMEM), dK += dS^T Q (A = the dS tile, K-major),
+//   dQ^T = K^T dS^T (B = the same tile, MN-major) -> TMEM [128,256)
+//   dQ^T -> row-major staging in the chunk's Q/dO stage -> one bulk fp32
+//   reduction per token into a global accumulator.
+// TMEM holds one chunk at a time (S^T, dP^T, dV, dK fill all 512 columns);
+// S^T of the next chunk is issued right behind the current chunk's MMAs and
+// dP^T once the dQ^T columns have been read out.
 #include <math.h>
 
 #include "msa_device.cuh"
@@ -27,7 +33,7 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 448;   // w0 TMA(K,V) | w1 MMA | w2-5 gather | w6-9 dS | w10-13 dQ, dK/dV out
+constexpr int kWarps = 18;   // w0 TMA(K,V) | w1 MMA | w2-9 softmax | w10-13 gather | w14-17 dQ, dK/dV
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdParams {
@@ -50,35 +56,29 @@ struct BwdParams {
 
 template <int D>
 struct BwdSmem {
-    static constexpr int kStages = 4;                           // Q/dO ring
     static constexpr uint32_t kKV = 128u * D * 2u;              // one K or V tile
-    static constexpr uint32_t kHalf = 64u * D * 2u;             // Q or dO of one 64-row chunk
-    static constexpr uint32_t kK = 0, kV = kKV;
+    static constexpr uint32_t kHalf = 128u * D * 2u;            // Q or dO of one 128-row chunk
+    static constexpr uint32_t kK = 0, kV = kKV;                 // V right after K (d = 64 dQ^T reads on)
     static constexpr uint32_t kStage0 = 2 * kKV;                // stage s: Q at s*2*kHalf, dO after it
-    static constexpr uint32_t kDS = kStage0 + kStages * 2 * kHalf;   // 2 dS tiles (128 keys x 64 rows)
-    static constexpr uint32_t kDSTile = 128u * 64u * 2u;
-    static constexpr uint32_t kMeta = kDS + 2 * kDSTile;        // per stage {L2[64], D[64], cmax[64]}
-    static constexpr uint32_t kMetaStage = 64 * 4 * 2 + 64;
-    static constexpr uint32_t kBars = kMeta + kStages * kMetaStage;
-    static constexpr uint32_t kNumBars = 1 + 2 * kStages + 5 * 2 + 2;
+    static constexpr uint32_t kDS = kStage0 + 2 * 2 * kHalf;    // dS^T tile: 128 keys x 128 rows bf16
+    static constexpr uint32_t kDSBytes = 128u * 128u * 2u;
+    static constexpr uint32_t kMeta = kDS + kDSBytes;           // per stage {L2[128], D*scale[128], cm[128], flag}
+    static constexpr uint32_t kMetaStage = 128 * 4 * 2 + 128 + 16;
+    static constexpr uint32_t kBars = kMeta + 2 * kMetaStage;
+    static constexpr uint32_t kNumBars = 1 + 2 + 2 + 5;
     static constexpr uint32_t kTotal = kBars + kNumBars * 8 + 8;
+    static_assert(kTotal <= 232448, "shared memory per CTA");
     static_assert(2 * 128 * (D * 4 + 16) <= kMeta - kStage0, "dK/dV staging must fit the stage and dS area");
+    static_assert(128u * D * 4u <= 2 * kHalf, "dQ staging must fit one stage");
 };
 
-// Work per item: the 64-row chunks (64/G tokens x G heads) of the item's
-// queries, software-pipelined over two TMEM buffer sets:
-//   MMA:      S^T(c), dP^T(c) -> buffer c&1      (issued two chunks ahead)
-//   softmax:  P^T, dS^T (bf16) into the same buffer, dS^T into smem tile c&1
-//   MMA:      dV += P^T dO, dK += dS^T Q, dQ^T = K^T dS^T (into dP^T's columns)
-//   epilogue: dQ^T -> this chunk's Q/dO stage (row-major) -> bulk fp32
-//             reduction per token; the stage is then free for chunk c+4.
+// Work per item: chunks c of 128 query rows, token-major (row = t*G + hh).
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kWarps * 32, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 BwdParams p)
 {
     using SM = BwdSmem<D>;
-    constexpr int kS = SM::kStages;
     constexpr uint32_t kKV = SM::kKV, kHalf = SM::kHalf;
     constexpr int kSlabs = D / 64;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -102,37 +102,32 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint8_t* v_tile = smem + SM::kV;
     uint64_t* bars = (uint64_t*)(smem + SM::kBars);
     uint64_t* kv_full = bars;
-    uint64_t* st_full = bars + 1;           // [kS] producers -> MMA
-    uint64_t* st_empty = st_full + kS;      // [kS] dQ epilogue -> producers
-    uint64_t* s_full = st_empty + kS;       // [2] MMA -> softmax
-    uint64_t* p_full = s_full + 2;          // [2] softmax -> MMA
-    uint64_t* ds_empty = p_full + 2;        // [2] MMA (dQ^T read dS tile) -> softmax
-    uint64_t* dq_full = ds_empty + 2;       // [2] MMA -> dQ epilogue
-    uint64_t* dq_empty = dq_full + 2;       // [2] dQ epilogue (TMEM drained) -> MMA
-    uint64_t* kv_done = dq_empty + 2;
-    uint64_t* fin = kv_done + 1;
+    uint64_t* st_full = bars + 1;           // [2] gather -> MMA, softmax
+    uint64_t* st_empty = st_full + 2;       // [2] dQ epilogue (staging read) -> gather
+    uint64_t* s_full = st_empty + 2;        // MMA -> softmax (S^T, dP^T; earlier MMAs done)
+    uint64_t* p_full = s_full + 1;          // softmax -> MMA (P^T in TMEM, dS^T in smem)
+    uint64_t* dq_full = p_full + 1;         // MMA -> dQ epilogue (every MMA of the chunk done)
+    uint64_t* dq_drained = dq_full + 1;     // dQ epilogue (TMEM read) -> MMA
+    uint64_t* fin = dq_drained + 1;
     uint32_t* tmem_hold = (uint32_t*)(bars + SM::kNumBars);
     volatile uint32_t* abort_flag = tmem_hold + 1;
     const WaitCtx wc{p.status, abort_flag, MSA_WAIT_LIMIT_NS};
 
     auto q_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kHalf; };
     auto do_stage = [&](int s) { return smem + SM::kStage0 + (uint32_t)s * 2u * kHalf + kHalf; };
-    auto ds_tile = [&](int bb) { return smem + SM::kDS + (uint32_t)bb * SM::kDSTile; };
+    uint8_t* ds_tile = smem + SM::kDS;
     auto meta_l2 = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage); };
-    auto meta_d = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage + 256); };
-    auto meta_cm = [&](int s) { return (int8_t*)(smem + SM::kMeta + s * SM::kMetaStage + 512); };
+    auto meta_d = [&](int s) { return (float*)(smem + SM::kMeta + s * SM::kMetaStage + 512); };
+    auto meta_cm = [&](int s) { return (int8_t*)(smem + SM::kMeta + s * SM::kMetaStage + 1024); };
+    auto meta_flag = [&](int s) { return (int*)(smem + SM::kMeta + s * SM::kMetaStage + 1152); };
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        for (int s = 0; s < kS; ++s) { mbar_init(&st_full[s], 128); mbar_init(&st_empty[s], 1); }
-        for (int bb = 0; bb < 2; ++bb) {
-            mbar_init(&s_full[bb], 1);
-            mbar_init(&p_full[bb], 128);
-            mbar_init(&ds_empty[bb], 1);
-            mbar_init(&dq_full[bb], 1);
-            mbar_init(&dq_empty[bb], 128);
-        }
-        mbar_init(kv_done, 1);
+        for (int s = 0; s < 2; ++s) { mbar_init(&st_full[s], 128); mbar_init(&st_empty[s], 1); }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 256);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_drained, 128);
         mbar_init(fin, 1);
         *abort_flag = 0u;
         fence_mbar_init();
@@ -142,10 +137,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_hold;
-    // TMEM columns: buffer bb at bb*128: S^T/P^T [0,64), dP^T/dS^T/dQ^T [64,128);
-    // dV at 256, dK at 256 + D.
-    auto tS = [&](int bb) { return tmem + (uint32_t)bb * 128u; };
-    auto tdP = [&](int bb) { return tmem + (uint32_t)bb * 128u + 64u; };
+    // TMEM columns: S^T / P^T [0,128), dP^T / dQ^T [128,256), dV at 256, dK at 256 + D.
+    const uint32_t tS = tmem, tdP = tmem + 128u;
     const uint32_t tdV = tmem + 256u, tdK = tmem + 256u + D;
 
     if (warp == 0) {
@@ -162,141 +155,107 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t idSS = idesc_bf16(128, 64, false, false);    // S^T, dP^T
-            constexpr uint32_t idKV = idesc_bf16(128, D, false, true);      // dV, dK (A in TMEM)
-            constexpr uint32_t idQT = idesc_bf16(128, 64, true, true);      // dQ^T (M = d, padded to 128)
-            const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile);
-            auto issue_pre = [&](int c) -> bool {   // S^T(c), dP^T(c)
-                const int s = c % kS, bb = c & 1;
-                if (!mbar_wait(&st_full[s], (uint32_t)(c / kS) & 1u, wc, code0 + 1)) return false;
-                if (c >= 2 && !mbar_wait(&dq_empty[bb], (uint32_t)((c - 2) >> 1) & 1u, wc, code0 + 2))
-                    return false;
-                tc_fence_after();
-                const uint32_t qa = smem_u32(q_stage(s)), oa = smem_u32(do_stage(s));
-                // S^T and dP^T are independent accumulation chains: interleaving
-                // their K-steps keeps more MMAs in flight than one chain at a time
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    umma_ss(tS(bb), desc_kmajor(ka, 128, kk * 16), desc_kmajor(qa, 64, kk * 16), idSS,
-                            kk > 0 ? 1u : 0u);
-                    umma_ss(tdP(bb), desc_kmajor(va, 128, kk * 16), desc_kmajor(oa, 64, kk * 16), idSS,
-                            kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&s_full[bb]);
-                return true;
-            };
+            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);    // S^T, dP^T (N = 128 rows)
+            constexpr uint32_t idKV = idesc_bf16(128, D, false, true);      // dV, dK (N = d)
+            constexpr uint32_t idQT = idesc_bf16(128, 128, true, true);     // dQ^T (M = d, padded to 128)
+            const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile), dsa = smem_u32(ds_tile);
             bool ok = mbar_wait(kv_full, 0, wc, code0 + 0);
-            if (ok && nchunks > 0) ok = issue_pre(0);
-            if (ok && nchunks > 1) ok = issue_pre(1);
             for (int c = 0; ok && c < nchunks; ++c) {
-                const int s = c % kS, bb = c & 1;
-                if (!mbar_wait(&p_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 3)) break;
+                const int s = c & 1;
+                if (!mbar_wait(&st_full[s], (uint32_t)(c >> 1) & 1u, wc, code0 + 1)) break;
                 tc_fence_after();
                 const uint32_t qa = smem_u32(q_stage(s)), oa = smem_u32(do_stage(s));
-                const uint32_t dsa = smem_u32(ds_tile(bb));
+                // S^T(c): its columns held P^T(c-1), which the dV MMAs issued
+                // before this point have consumed (MMAs run in issue order)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {   // K = 64 rows; dV and dK chains interleaved
-                    umma_ts(tdV, tS(bb) + kk * 8, desc_mnmajor(oa, 64, kk * 16), idKV,
-                            (c > 0 || kk > 0) ? 1u : 0u);
-                    umma_ts(tdK, tdP(bb) + kk * 8, desc_mnmajor(qa, 64, kk * 16), idKV,
-                            (c > 0 || kk > 0) ? 1u : 0u);
-                }
-                // dQ^T = K^T dS^T over the 128 keys; with d = 64 the second half
-                // of the M = 128 tile reads the V tile and lands in TMEM lanes
-                // nobody reads.
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ss(tdP(bb), desc_mnmajor(ka, 128, kk * 16), desc_mnmajor(dsa, 128, kk * 16), idQT,
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tS, desc_kmajor(ka, 128, kk * 16), desc_kmajor(qa, 128, kk * 16), idS,
                             kk > 0 ? 1u : 0u);
-                umma_commit(&ds_empty[bb]);
-                umma_commit(&dq_full[bb]);
-                if (c + 2 < nchunks) ok = issue_pre(c + 2);
+                // dP^T(c) overwrites dQ^T(c-1): wait until it has been read out
+                if (c > 0 && !mbar_wait(dq_drained, (uint32_t)(c - 1) & 1u, wc, code0 + 2)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tdP, desc_kmajor(va, 128, kk * 16), desc_kmajor(oa, 128, kk * 16), idS,
+                            kk > 0 ? 1u : 0u);
+                umma_commit(s_full);
+                if (!mbar_wait(p_full, (uint32_t)c & 1u, wc, code0 + 3)) break;
+                tc_fence_after();
+                // dV, dK (K = 128 rows) and dQ^T (K = 128 keys): three independent
+                // accumulation chains, interleaved
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t pcol = kk < 4 ? (uint32_t)kk * 8u : 64u + (uint32_t)(kk - 4) * 8u;
+                    umma_ts(tdV, tS + pcol, desc_mnmajor(oa, 128, kk * 16), idKV, (c > 0 || kk > 0) ? 1u : 0u);
+                    umma_ss(tdK, desc_kmajor(dsa, 128, kk * 16), desc_mnmajor(qa, 128, kk * 16), idKV,
+                            (c > 0 || kk > 0) ? 1u : 0u);
+                    umma_ss(tdP, desc_mnmajor(ka, 128, kk * 16), desc_mnmajor(dsa, 128, kk * 16), idQT,
+                            kk > 0 ? 1u : 0u);
+                }
+                umma_commit(dq_full);
             }
-            umma_commit(kv_done);
             umma_commit(fin);
             mbar_drain(fin, 0);
         }
-    } else if (warp < 6) {
-        // ---------------- gather Q, dO (64 rows) and per-row metadata ----------------
-        const int tid = threadIdx.x - 64;
-        constexpr int kPieces = 64 * D / 8;
-        constexpr int kRowPieces = D / 8;
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % kS;
-            const uint32_t su = (uint32_t)(c / kS);
-            if (su > 0 && !mbar_wait(&st_empty[s], (su - 1) & 1u, wc, code0 + 4)) break;
-            const uint32_t qs = smem_u32(q_stage(s)), os = smem_u32(do_stage(s));
-#pragma unroll 4
-            for (int it = 0; it < kPieces / 128; ++it) {
-                const int piece = it * 128 + tid;
-                const int row = piece / kRowPieces, ch = piece % kRowPieces;
-                const int t = row >> p.lgG, hh = row & (G - 1);
-                const int jj = c * p.tpc + t;
-                const bool valid = jj < count;
-                const int i = valid ? toks[jj] : 0;
-                const int64_t off = (((int64_t)b * p.T + i) * p.Hq + g * G + hh) * D + ch * 8;
-                const uint32_t dst = sw128_offset(row, ch & 7, ch >> 3, 64);
-                cp_async_16(qs + dst, p.q + off, valid ? 16u : 0u);
-                cp_async_16(os + dst, p.dout + off, valid ? 16u : 0u);
-            }
-            if (tid < 64) {
-                const int row = tid;
-                const int t = row >> p.lgG, hh = row & (G - 1), h = g * G + hh;
-                const int jj = c * p.tpc + t;
-                const bool valid = jj < count;
-                const int i = valid ? toks[jj] : 0;
-                const int64_t lrow = ((int64_t)b * p.Hq + h) * p.T + i;
-                meta_l2(s)[row] = valid ? p.lse[lrow] * kLog2e : 0.f;
-                meta_d(s)[row] = valid ? p.dsum[lrow] : 0.f;
-                meta_cm(s)[row] = (int8_t)(valid ? (((i >> 7) == n) ? (i & 127) : 127) : -1);
-            }
-            cp_async_commit();
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            mbar_arrive(&st_full[s]);
-        }
-        cp_async_wait<0>();
     } else if (warp < 10) {
         // ---------------- P^T, dS^T (one TMEM lane = one key) ----------------
-        const int jl = ((warp & 3) << 5) | lane;   // key within the block
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        // Two warps per TMEM lane quarter: warp half hf takes rows [64 hf, 64 hf + 64).
+        const int qd4 = warp & 3, hf = (warp - 2) >> 2;
+        const int jl = (qd4 << 5) | lane;   // key within the block
+        const uint32_t lane_base = (uint32_t)(qd4 * 32);
+        const uint32_t dsa = smem_u32(ds_tile);
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c % kS, bb = c & 1;
-            bool ok = mbar_wait(&s_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 5);
-            if (ok && c >= 2) ok = mbar_wait(&ds_empty[bb], (uint32_t)((c - 2) >> 1) & 1u, wc, code0 + 6);
+            const int s = c & 1;
+            // s_full(c) also means dK(c-1) and dQ^T(c-1) have read the dS tile;
+            // st_full (long complete by then) orders the gather's metadata stores
+            bool ok = mbar_wait(s_full, (uint32_t)c & 1u, wc, code0 + 5);
+            if (ok) ok = mbar_wait(&st_full[s], (uint32_t)(c >> 1) & 1u, wc, code0 + 6);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const float* L2 = meta_l2(s);
             const float* Dv = meta_d(s);
             const int8_t* cm = meta_cm(s);
-            const uint32_t aS = tmem_addr(tS(bb), lane_base, 0), aP = tmem_addr(tdP(bb), lane_base, 0);
-            const uint32_t dsa = smem_u32(ds_tile(bb));
+            const bool masked = *(volatile int*)meta_flag(s) != 0;   // chunk holds block-n queries
 #pragma unroll
-            for (int piece = 0; piece < 2; ++piece) {
+            for (int pp = 0; pp < 2; ++pp) {
+                const int piece = 2 * hf + pp;   // rows piece*32 .. +31
                 uint32_t sv[32], dv[32], pk[16], dk[16];
-                tmem_ld32(aS + piece * 32, sv);
-                tmem_ld32(aP + piece * 32, dv);
+                tmem_ld32(tmem_addr(tS, lane_base, (uint32_t)piece * 32u), sv);
+                tmem_ld32(tmem_addr(tdP, lane_base, (uint32_t)piece * 32u), dv);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int r0 = piece * 32 + 2 * e, r1 = r0 + 1;
-                    const float p0 = jl <= (int)cm[r0]
-                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e]), p.c1, -L2[r0]))
-                                         : 0.f;
-                    const float p1 = jl <= (int)cm[r1]
-                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), p.c1, -L2[r1]))
-                                         : 0.f;
-                    const float d0 = p0 * (__uint_as_float(dv[2 * e]) - Dv[r0]) * p.scale;
-                    const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - Dv[r1]) * p.scale;
-                    pk[e] = pack_bf16x2(p0, p1);
-                    dk[e] = pack_bf16x2(d0, d1);
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const int r0 = piece * 32 + 4 * e4;
+                    const float4 l4 = *reinterpret_cast<const float4*>(L2 + r0);
+                    const float4 d4 = *reinterpret_cast<const float4*>(Dv + r0);
+                    float pr[4];
+                    pr[0] = ex2_approx(fmaf(__uint_as_float(sv[4 * e4 + 0]), p.c1, -l4.x));
+                    pr[1] = ex2_approx(fmaf(__uint_as_float(sv[4 * e4 + 1]), p.c1, -l4.y));
+                    pr[2] = ex2_approx(fmaf(__uint_as_float(sv[4 * e4 + 2]), p.c1, -l4.z));
+                    pr[3] = ex2_approx(fmaf(__uint_as_float(sv[4 * e4 + 3]), p.c1, -l4.w));
+                    if (masked) {
+                        const uint32_t c4 = *reinterpret_cast<const uint32_t*>(cm + r0);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (jl > (int)(int8_t)(c4 >> (8 * u))) pr[u] = 0.f;
+                    }
+                    // dS = P (dP - D) scale, as P (dP scale - D scale)
+                    const float s0 = pr[0] * fmaf(__uint_as_float(dv[4 * e4 + 0]), p.scale, -d4.x);
+                    const float s1 = pr[1] * fmaf(__uint_as_float(dv[4 * e4 + 1]), p.scale, -d4.y);
+                    const float s2 = pr[2] * fmaf(__uint_as_float(dv[4 * e4 + 2]), p.scale, -d4.z);
+                    const float s3 = pr[3] * fmaf(__uint_as_float(dv[4 * e4 + 3]), p.scale, -d4.w);
+                    pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+                    pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
+                    dk[2 * e4] = pack_bf16x2(s0, s1);
+                    dk[2 * e4 + 1] = pack_bf16x2(s2, s3);
                 }
-                tmem_st16(aS + piece * 16, pk);   // P^T over S^T columns already read
-                tmem_st16(aP + piece * 16, dk);   // dS^T over dP^T columns already read
-                // dS^T row jl (rows piece*32 .. +31) into the MN-major dS tile
+                // P^T rows piece*32.. over S^T columns this warp has already read
+                tmem_st16(tmem_addr(tS, lane_base, (uint32_t)(64 * hf + 16 * pp)), pk);
+                // dS^T row jl, query rows piece*32 .. +31 (slab piece/2 of the tile)
 #pragma unroll
                 for (int qd = 0; qd < 4; ++qd) {
-                    const uint32_t addr = dsa + sw128_offset((uint32_t)jl, (uint32_t)(piece * 4 + qd), 0, 128);
+                    const uint32_t addr =
+                        dsa + sw128_offset((uint32_t)jl, (uint32_t)((piece & 1) * 4 + qd), (uint32_t)(piece >> 1), 128);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * qd]),
                                  "r"(dk[4 * qd + 1]), "r"(dk[4 * qd + 2]), "r"(dk[4 * qd + 3])
                                  : "memory");
@@ -305,55 +264,122 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tmem_st_wait();
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&p_full[bb]);
+            mbar_arrive(p_full);
         }
+    } else if (warp < 14) {
+        // ---------------- gather Q, dO (128 rows) and per-row metadata ----------------
+        // Thread tid copies 16-byte column ch of rows r0, r0 + kRowStep, ...:
+        // two neighbouring rows per warp and instruction, each row whole.  The
+        // next chunk's token ids and metadata are loaded while this chunk's
+        // copies are in flight.
+        const int tid = threadIdx.x - 320;
+        constexpr int kRowPieces = D / 8;
+        constexpr int kRowStep = 128 / kRowPieces;
+        const int ch = tid % kRowPieces, r0 = tid / kRowPieces;
+        int tk[kRowPieces];          // token of each of this thread's rows (-1: past the end)
+        int m_tok = -1;              // token of metadata row tid
+        float m_l2 = 0.f, m_d = 0.f;
+        auto fetch = [&](int c) {
+#pragma unroll
+            for (int it = 0; it < kRowPieces; ++it) {
+                const int jj = c * p.tpc + ((r0 + it * kRowStep) >> p.lgG);
+                tk[it] = jj < count ? __ldg(toks + jj) : -1;
+            }
+            const int jj = c * p.tpc + (tid >> p.lgG);
+            m_tok = jj < count ? __ldg(toks + jj) : -1;
+            if (m_tok >= 0) {
+                const int64_t lrow = ((int64_t)b * p.Hq + g * G + (tid & (G - 1))) * p.T + m_tok;
+                m_l2 = __ldg(p.lse + lrow) * kLog2e;
+                m_d = __ldg(p.dsum + lrow) * p.scale;
+            } else {
+                m_l2 = 0.f;
+                m_d = 0.f;
+            }
+        };
+        fetch(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const uint32_t su = (uint32_t)(c >> 1);
+            if (su > 0 && !mbar_wait(&st_empty[s], (su - 1) & 1u, wc, code0 + 4)) break;
+            const uint32_t qs = smem_u32(q_stage(s)), os = smem_u32(do_stage(s));
+#pragma unroll
+            for (int it = 0; it < kRowPieces; ++it) {
+                const int row = r0 + it * kRowStep;
+                const bool valid = tk[it] >= 0;
+                const int64_t off =
+                    (((int64_t)b * p.T + (valid ? tk[it] : 0)) * p.Hq + g * G + (row & (G - 1))) * D + ch * 8;
+                const uint32_t dst = sw128_offset((uint32_t)row, (uint32_t)(ch & 7), (uint32_t)(ch >> 3), 128);
+                cp_async_16(qs + dst, p.q + off, valid ? 16u : 0u);
+                cp_async_16(os + dst, p.dout + off, valid ? 16u : 0u);
+            }
+            cp_async_commit();
+            {
+                // rows past the item's end read as zeros with L2 = D = 0: their P is
+                // finite and meets only zero dO, and dP - D = 0, so they add nothing
+                const bool diag = m_tok >= 0 && (m_tok >> 7) == n;
+                meta_l2(s)[tid] = m_l2;
+                meta_d(s)[tid] = m_d;
+                meta_cm(s)[tid] = (int8_t)(diag ? (m_tok & 127) : 127);
+                // token lists are ascending, so block-n queries come first
+                if (tid == 0) *meta_flag(s) = diag ? 1 : 0;
+            }
+            if (c + 1 < nchunks) fetch(c + 1);
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&st_full[s]);
+        }
+        cp_async_wait<0>();
     } else {
         // ---------------- dQ partials out; dK, dV partials at the end ----------------
         const int r = ((warp & 3) << 5) | lane;    // TMEM lane = head-dim index of dQ^T
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        const int tid = threadIdx.x - 320;
+        const int tid = threadIdx.x - 448;
         const uint32_t tok_bytes = (uint32_t)G * D * 4u;
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c % kS, bb = c & 1;
-            ok = bar_and_sync(1, 128, mbar_wait(&dq_full[bb], (uint32_t)(c >> 1) & 1u, wc, code0 + 7));
+            const int s = c & 1;
+            const int ntok = min(p.tpc, count - c * p.tpc);
+            const int my_tok = tid < ntok ? __ldg(toks + c * p.tpc + tid) : 0;   // loaded before the wait
+            ok = bar_and_sync(1, 128, mbar_wait(dq_full, (uint32_t)c & 1u, wc, code0 + 7));
             if (!ok) break;   // all four warps leave together: none is left at a barrier below
             tc_fence_after();
-            // dQ^T[r][row] for the chunk's 64 rows -> row-major staging in this
+            // dQ^T[r][row] for the chunk's 128 rows -> row-major staging in this
             // chunk's Q/dO stage (32 consecutive floats per warp store)
             const uint32_t stg = smem_u32(q_stage(s));
-            uint32_t v[64];
-            tmem_ld32(tmem_addr(tdP(bb), lane_base, 0), v);
-            tmem_ld32(tmem_addr(tdP(bb), lane_base, 32), v + 32);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&dq_empty[bb]);     // TMEM columns free for chunk c+2
-            if (r < D) {
 #pragma unroll
-                for (int e = 0; e < 64; ++e)
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + ((uint32_t)e * D + (uint32_t)r) * 4u),
-                                 "r"(v[e])
-                                 : "memory");
+            for (int hx = 0; hx < 2; ++hx) {
+                uint32_t v[64];
+                tmem_ld32(tmem_addr(tdP, lane_base, (uint32_t)hx * 64u), v);
+                tmem_ld32(tmem_addr(tdP, lane_base, (uint32_t)hx * 64u + 32u), v + 32);
+                tmem_ld_wait();
+                if (hx == 1) {
+                    tc_fence_before();
+                    mbar_arrive(dq_drained);     // TMEM columns free for dP^T(c+1)
+                }
+                if (r < D) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + ((uint32_t)(hx * 64 + e) * D + (uint32_t)r) * 4u),
+                                     "r"(v[e])
+                                     : "memory");
+                }
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
-            const int ntok = min(p.tpc, count - c * p.tpc);
-            for (int t = tid; t < ntok; t += 128) {
-                const int i = toks[c * p.tpc + t];
+            if (tid < ntok)   // one token per thread: at most 128 tokens per chunk
                 asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                                 p.dqacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D),
-                             "r"(stg + (uint32_t)t * tok_bytes), "r"(tok_bytes)
+                                 p.dqacc + (((int64_t)b * p.T + my_tok) * p.Hq + g * G) * D),
+                             "r"(stg + (uint32_t)tid * tok_bytes), "r"(tok_bytes)
                              : "memory");
-            }
             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             named_bar_sync(1, 128);
             if (tid == 0) mbar_arrive(&st_empty[s]);
         }
-        if (ok) ok = mbar_wait(kv_done, 0, wc, code0 + 8);
-        if (__all_sync(0xffffffffu, ok)) {
-            // This item's dK, dV partials (lane = key) -> padded staging in the
-            // now idle stage and dS area -> one bulk fp32 reduction per key row.
+        if (ok) {
+            // The last dq_full covers every MMA of the item.  Its dK, dV partials
+            // (lane = key) -> padded staging in the now idle stage and dS area ->
+            // one bulk fp32 reduction per key row.
             tc_fence_after();
             const uint32_t row_stride = D * 4u + 16u;
             const uint32_t stg = smem_u32(smem + SM::kStage0);
@@ -432,7 +458,7 @@ __global__ void __launch_bounds__(256) bwd_dsum_kernel(const __nv_bfloat16* __re
     }
 }
 
-// fp32 dQ accumulator -> bf16, 8 elements per thread.
+// fp32 accumulator -> bf16, 8 elements per thread.
 __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __restrict__ acc,
                                                              __nv_bfloat16* __restrict__ dq, int64_t n8)
 {
@@ -471,7 +497,7 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     BwdParams p;
     p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
     p.lgG = 31 - __builtin_clz((unsigned)pr.G);
-    p.tpc = 64 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;   // 64-row chunks
+    p.tpc = 128 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;   // 128-row chunks
     p.c1 = pr.scale * kLog2e;
     p.scale = pr.scale;
     p.q = (const __nv_bfloat16*)q;
@@ -492,7 +518,7 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
                                   (int)smem)) != cudaSuccess)
         return e;
     trace_begin(kTraceBwdMain, st);
-    bwd_main_kernel<D><<<(unsigned)(p.per_group * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+    bwd_main_kernel<D><<<(unsigned)(p.per_group * pr.B * pr.Hkv), kWarps * 32, smem, st>>>(tm_k, tm_v, p);
     trace_end(kTraceBwdMain, st);
     const int64_t n8 = pr.rows_q() * D / 8;
     bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dqacc, (__nv_bfloat16*)dq, n8);
