@@ -20,8 +20,9 @@
 //                  dS^T = P^T (dP^T scale - D scale) (bf16) into a shared-memory tile
 //   dV += P^T dO (A from TMEM), dK += dS^T Q (A = the dS tile, K-major),
 //   dQ^T = K^T dS^T (B = the same tile, MN-major) -> TMEM [128,256)
-//   dQ^T -> row-major staging in the chunk's Q/dO stage -> one bulk fp32
-//   reduction per token into a global accumulator.
+//   dQ^T -> row-major staging in the chunk's Q/dO stage, a quarter (32 rows)
+//   at a time -> one bulk fp32 reduction per token into a global accumulator,
+//   issued by warp 0 so that the staging warps never wait on the reduction.
 // TMEM holds one chunk at a time (S^T, dP^T, dV, dK fill all 512 columns);
 // S^T of the next chunk is issued right behind the current chunk's MMAs and
 // dP^T once the dQ^T columns have been read out.
@@ -33,7 +34,7 @@
 namespace msa {
 namespace {
 
-constexpr int kWarps = 18;   // w0 TMA(K,V) | w1 MMA | w2-9 softmax | w10-13 gather | w14-17 dQ, dK/dV
+constexpr int kWarps = 18;   // w0 TMA(K,V), dQ reductions | w1 MMA | w2-9 softmax | w10-13 gather | w14-17 dQ, dK/dV
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdParams {
@@ -65,7 +66,7 @@ struct BwdSmem {
     static constexpr uint32_t kMeta = kDS + kDSBytes;           // per stage {L2[128], D*scale[128], cm[128], flag}
     static constexpr uint32_t kMetaStage = 128 * 4 * 2 + 128 + 16;
     static constexpr uint32_t kBars = kMeta + 2 * kMetaStage;
-    static constexpr uint32_t kNumBars = 1 + 2 + 2 + 5;
+    static constexpr uint32_t kNumBars = 1 + 2 + 2 + 5 + 8;
     static constexpr uint32_t kTotal = kBars + kNumBars * 8 + 8;
     static_assert(kTotal <= 232448, "shared memory per CTA");
     static_assert(2 * 128 * (D * 4 + 16) <= kMeta - kStage0, "dK/dV staging must fit the stage and dS area");
@@ -109,6 +110,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t* dq_full = p_full + 1;         // MMA -> dQ epilogue (every MMA of the chunk done)
     uint64_t* dq_drained = dq_full + 1;     // dQ epilogue (TMEM read) -> MMA
     uint64_t* fin = dq_drained + 1;
+    uint64_t* stg_full = fin + 1;           // [2][4] dQ epilogue (quarter staged) -> warp 0
     uint32_t* tmem_hold = (uint32_t*)(bars + SM::kNumBars);
     volatile uint32_t* abort_flag = tmem_hold + 1;
     const WaitCtx wc{p.status, abort_flag, MSA_WAIT_LIMIT_NS};
@@ -129,6 +131,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(dq_full, 1);
         mbar_init(dq_drained, 128);
         mbar_init(fin, 1);
+        for (int x = 0; x < 8; ++x) mbar_init(&stg_full[x], 128);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -152,6 +155,48 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             mbar_drain(kv_full, 0);
         }
+        __syncwarp();
+        // ---------------- dQ bulk reductions ----------------
+        // Quarter qq of chunk c holds tokens [qq*qt, qq*qt + qt) of the chunk;
+        // lane l reduces token qq*qt + l.  Stage sets alternate with the chunk
+        // parity, so a set is reused only after this warp released its stage.
+        const int qt = p.tpc >> 2;
+        const uint32_t tok_bytes = (uint32_t)G * D * 4u;
+        int tq[4];
+        auto load_tokens = [&](int c) {
+            const int ntok = min(p.tpc, count - c * p.tpc);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const int t = qq * qt + lane;
+                tq[qq] = (lane < qt && t < ntok) ? __ldg(toks + c * p.tpc + t) : -1;
+            }
+        };
+        load_tokens(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const uint32_t stg = smem_u32(q_stage(s));
+            bool ok = true;
+            bool issued = false;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                ok = mbar_wait(&stg_full[s * 4 + qq], (uint32_t)(c >> 1) & 1u, wc, code0 + 9);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                if (tq[qq] >= 0) {
+                    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                                     p.dqacc + (((int64_t)b * p.T + tq[qq]) * p.Hq + g * G) * D),
+                                 "r"(stg + (uint32_t)(qq * qt + lane) * tok_bytes), "r"(tok_bytes)
+                                 : "memory");
+                    issued = true;
+                }
+            }
+            if (issued) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            if (!ok) break;
+            if (c + 1 < nchunks) load_tokens(c + 1);
+            if (issued) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&st_empty[s]);   // staging read: the stage may be refilled
+        }
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
@@ -277,16 +322,20 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         constexpr int kRowStep = 128 / kRowPieces;
         const int ch = tid % kRowPieces, r0 = tid / kRowPieces;
         int tk[kRowPieces];          // token of each of this thread's rows (-1: past the end)
-        int m_tok = -1;              // token of metadata row tid
+        int m_tok = -1, m_tok_next = -1;   // token of metadata row tid: this chunk, the next
         float m_l2 = 0.f, m_d = 0.f;
-        auto fetch = [&](int c) {
+        auto row_tokens = [&](int c) {
 #pragma unroll
             for (int it = 0; it < kRowPieces; ++it) {
                 const int jj = c * p.tpc + ((r0 + it * kRowStep) >> p.lgG);
                 tk[it] = jj < count ? __ldg(toks + jj) : -1;
             }
+        };
+        auto meta_token = [&](int c) {
             const int jj = c * p.tpc + (tid >> p.lgG);
-            m_tok = jj < count ? __ldg(toks + jj) : -1;
+            return (c < nchunks && jj < count) ? __ldg(toks + jj) : -1;
+        };
+        auto meta_values = [&]() {   // for m_tok, loaded one chunk before its use
             if (m_tok >= 0) {
                 const int64_t lrow = ((int64_t)b * p.Hq + g * G + (tid & (G - 1))) * p.T + m_tok;
                 m_l2 = __ldg(p.lse + lrow) * kLog2e;
@@ -296,7 +345,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 m_d = 0.f;
             }
         };
-        fetch(0);
+        row_tokens(0);
+        m_tok = meta_token(0);
+        meta_values();
+        m_tok_next = meta_token(1);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
             const uint32_t su = (uint32_t)(c >> 1);
@@ -323,7 +375,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 // token lists are ascending, so block-n queries come first
                 if (tid == 0) *meta_flag(s) = diag ? 1 : 0;
             }
-            if (c + 1 < nchunks) fetch(c + 1);
+            // next chunk: its row tokens, the metadata of its row tid (whose token
+            // arrived during this chunk), and the token of the chunk after it
+            if (c + 1 < nchunks) {
+                row_tokens(c + 1);
+                m_tok = m_tok_next;
+                meta_values();
+                m_tok_next = meta_token(c + 2);
+            }
             cp_async_wait<0>();
             fence_proxy_async_smem();
             mbar_arrive(&st_full[s]);
@@ -333,49 +392,40 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // ---------------- dQ partials out; dK, dV partials at the end ----------------
         const int r = ((warp & 3) << 5) | lane;    // TMEM lane = head-dim index of dQ^T
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
-        const int tid = threadIdx.x - 448;
-        const uint32_t tok_bytes = (uint32_t)G * D * 4u;
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
-            const int ntok = min(p.tpc, count - c * p.tpc);
-            const int my_tok = tid < ntok ? __ldg(toks + c * p.tpc + tid) : 0;   // loaded before the wait
-            ok = bar_and_sync(1, 128, mbar_wait(dq_full, (uint32_t)c & 1u, wc, code0 + 7));
-            if (!ok) break;   // all four warps leave together: none is left at a barrier below
+            ok = mbar_wait(dq_full, (uint32_t)c & 1u, wc, code0 + 7);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
             // dQ^T[r][row] for the chunk's 128 rows -> row-major staging in this
-            // chunk's Q/dO stage (32 consecutive floats per warp store)
+            // chunk's Q/dO stage (32 consecutive floats per warp store), handed
+            // to warp 0 a quarter at a time
             const uint32_t stg = smem_u32(q_stage(s));
 #pragma unroll
-            for (int hx = 0; hx < 2; ++hx) {
-                uint32_t v[64];
-                tmem_ld32(tmem_addr(tdP, lane_base, (uint32_t)hx * 64u), v);
-                tmem_ld32(tmem_addr(tdP, lane_base, (uint32_t)hx * 64u + 32u), v + 32);
+            for (int qq = 0; qq < 4; ++qq) {
+                uint32_t v[32];
+                tmem_ld32(tmem_addr(tdP, lane_base, (uint32_t)qq * 32u), v);
                 tmem_ld_wait();
-                if (hx == 1) {
+                if (qq == 3) {
                     tc_fence_before();
                     mbar_arrive(dq_drained);     // TMEM columns free for dP^T(c+1)
                 }
                 if (r < D) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + ((uint32_t)(hx * 64 + e) * D + (uint32_t)r) * 4u),
+                    for (int e = 0; e < 32; ++e)
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(stg + ((uint32_t)(qq * 32 + e) * D + (uint32_t)r) * 4u),
                                      "r"(v[e])
                                      : "memory");
                 }
+                fence_proxy_async_smem();
+                mbar_arrive(&stg_full[s * 4 + qq]);
             }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (tid < ntok)   // one token per thread: at most 128 tokens per chunk
-                asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                                 p.dqacc + (((int64_t)b * p.T + my_tok) * p.Hq + g * G) * D),
-                             "r"(stg + (uint32_t)tid * tok_bytes), "r"(tok_bytes)
-                             : "memory");
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-            named_bar_sync(1, 128);
-            if (tid == 0) mbar_arrive(&st_empty[s]);
         }
+        // the dK/dV staging below reuses both stages: wait until warp 0's
+        // reductions have read the last chunks' dQ staging
+        for (int c = max(0, nchunks - 2); ok && c < nchunks; ++c)
+            ok = __all_sync(0xffffffffu, mbar_wait(&st_empty[c & 1], (uint32_t)(c >> 1) & 1u, wc, code0 + 8));
         if (ok) {
             // The last dq_full covers every MMA of the item.  Its dK, dV partials
             // (lane = key) -> padded staging in the now idle stage and dS area ->
