@@ -142,6 +142,21 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+# ---------------------------------------------------------------- ranks
+def combine_ranks(dist, world, device, ms, units):
+    """Whole-job figures of a weak-scaling run: each rank times its own batch,
+    the job takes as long as the slowest rank (max of ms) and does the work of
+    all ranks (sum of units).  One all-reduce each, same order on every rank."""
+    if world <= 1:
+        return ms, units
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
 # ---------------------------------------------------------------- CPU oracle timing
 def oracle_arrays(host):
     """float32 copies of the bf16 inputs (exact) for the oracle."""
@@ -300,6 +315,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    launches0 = msa.kernel_launches()
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -315,16 +331,14 @@ def main():
         step(d, ev)
     t_stop.record(stream)
     torch.cuda.synchronize()
+    launches = msa.kernel_launches() - launches0
     for kk in kernel_names:
         msa.set_kernel_events(kk, None, None)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     ms = t_start.elapsed_time(t_stop) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, f_job = combine_ranks(dist, world, dev, ms, f_step)
 
     phase = {"proxy_select": [], "fwd": [], "bwd": []}
     for ev in pev:
@@ -366,11 +380,8 @@ def main():
         b_.record(stream)
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b_) / e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * f_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+        e_ms, _ = combine_ranks(dist, world, dev, e_ms, f_step)
+        e2e = {"value": f_job / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     if world > 1:
@@ -380,7 +391,7 @@ def main():
         return
 
     peaks, peak_src = measured_peaks()
-    tflops = world * f_step / (ms * 1e-3) / 1e12
+    tflops = f_job / (ms * 1e-3) / 1e12
     tok_s = world * B * T / (ms * 1e-3)
     # dominant kernel of the step
     kf = {"proxy_select": f_proxy, "fwd_main": f_fwd, "bwd_main": f_bwd}
@@ -421,7 +432,7 @@ def main():
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 16 * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -173,10 +173,14 @@ cudaError_t launch_block_index(const Problem& pr, const int32_t* idx, const int3
     }
     dim3 g1(pr.nblk, BH);
     index_count_kernel<<<g1, 128, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, cnt, status);
+    count_launches(1);
     dim3 g2((pr.nblk + 31) / 32, BH), b2(32, 32);
     index_scan_kernel<<<g2, b2, 0, st>>>(cnt, tot, pr.nblk);
+    count_launches(1);
     index_ptr_kernel<<<BH, 1024, 0, st>>>(tot, ptr, pr.nblk);
+    count_launches(1);
     index_fill_kernel<<<g1, 128, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, cnt, ptr, tok);
+    count_launches(1);
     return cudaGetLastError();
 }
 

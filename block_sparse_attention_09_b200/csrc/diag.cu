@@ -159,12 +159,14 @@ cudaError_t launch_diag_umma(int mode, int N, int K, const void* A, const void* 
     if (e != cudaSuccess) return e;
     diag_umma_kernel<<<1, 128, smem, st>>>(mode, N, K, (const __nv_bfloat16*)A, (const __nv_bfloat16*)B,
                                            D, status);
+    count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_diag_wait(uint64_t limit_ns, uint32_t* status, cudaStream_t st)
 {
     diag_wait_kernel<<<1, 32, 0, st>>>(limit_ns, status);
+    count_launches(1);
     return cudaGetLastError();
 }
 

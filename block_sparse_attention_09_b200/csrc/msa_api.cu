@@ -3,6 +3,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/msa.h"
@@ -81,6 +82,10 @@ TraceEvents& trace_events()
     static thread_local TraceEvents t;
     return t;
 }
+
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 }  // namespace msa
 
@@ -250,6 +255,8 @@ const char* msa_strerror(int s)
     default: return "unknown status";
     }
 }
+
+uint64_t msa_kernel_launches(void) { return (uint64_t)msa::g_launches.load(std::memory_order_relaxed); }
 
 int msa_set_kernel_events(int kernel, void* start, void* stop)
 {

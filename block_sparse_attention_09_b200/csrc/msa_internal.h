@@ -61,6 +61,9 @@ struct TraceEvents {
     cudaEvent_t stop[kTraceCount] = {nullptr, nullptr, nullptr};
 };
 TraceEvents& trace_events();   // per host thread
+// Host-side count of kernel launches (msa_kernel_launches).
+void count_launches(unsigned n);
+
 inline void trace_begin(int k, cudaStream_t st)
 {
     TraceEvents& t = trace_events();

@@ -415,6 +415,7 @@ cudaError_t launch_variant(const Problem& pr, const CUtensorMap& tm_qp, const CU
     const unsigned grid = (unsigned)(pr.nblk * pr.B * pr.Hp);
     trace_begin(kTraceProxy, st);
     kern<<<grid, kThreads, smem, st>>>(tm_qp, tm_kp, p);
+    count_launches(1);
     trace_end(kTraceProxy, st);
     return cudaGetLastError();
 }

@@ -543,6 +543,7 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     const int64_t th = pr.rows_q() * (D / 8);
     bwd_dsum_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(
         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, dsum);
+    count_launches(1);
 
     BwdParams p;
     p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
@@ -569,12 +570,16 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
         return e;
     trace_begin(kTraceBwdMain, st);
     bwd_main_kernel<D><<<(unsigned)(p.per_group * pr.B * pr.Hkv), kWarps * 32, smem, st>>>(tm_k, tm_v, p);
+    count_launches(1);
     trace_end(kTraceBwdMain, st);
     const int64_t n8 = pr.rows_q() * D / 8;
     bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dqacc, (__nv_bfloat16*)dq, n8);
+    count_launches(1);
     const int64_t k8 = (int64_t)kv_elems / 8;
     bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dkacc, (__nv_bfloat16*)dk, k8);
+    count_launches(1);
     bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dvacc, (__nv_bfloat16*)dv, k8);
+    count_launches(1);
     return cudaGetLastError();
 }
 

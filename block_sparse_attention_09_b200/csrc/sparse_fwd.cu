@@ -498,6 +498,7 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     const int64_t th = nrows * (D / 8);
     fwd_norms_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(qb, kb, pr.B, pr.T, pr.Hq, pr.Hkv, qn,
                                                                      (uint32_t*)kmax);
+    count_launches(1);
 
     FwdParams p;
     p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
@@ -519,15 +520,18 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
         return e;
     trace_begin(kTraceFwdMain, st);
     fwd_main_kernel<D><<<(unsigned)(p.per_group * pr.B * pr.Hkv), kThreads, smem, st>>>(tm_k, tm_v, p);
+    count_launches(1);
     trace_end(kTraceFwdMain, st);
 
     const int64_t fth = (int64_t)pr.rows_q() * (D / 8);
     fwd_finalize_kernel<D><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(
         oacc, lacc, qn, kmax, pr.B, pr.T, pr.Hq, pr.Hkv, fabsf(pr.scale), (__nv_bfloat16*)o, lse, nflag,
         flags);
+    count_launches(1);
     fwd_fallback_kernel<D><<<148, 128, 0, st>>>(qb, kb, (const __nv_bfloat16*)v, idx, nsel, pr.B,
                                                 pr.T, pr.Hq, pr.Hkv, pr.topk, pr.scale, nflag, flags,
                                                 (__nv_bfloat16*)o, lse);
+    count_launches(1);
     return cudaGetLastError();
 }
 

@@ -60,6 +60,8 @@ def _load():
     lib.msa_diag_umma.argtypes = [I, I, I, P, P, P, P, P]
     lib.msa_diag_wait_timeout.argtypes = [U64, P, P]
     lib.msa_set_kernel_events.argtypes = [I, P, P]
+    lib.msa_kernel_launches.argtypes = []
+    lib.msa_kernel_launches.restype = U64
     for f in ("msa_proxy_select", "msa_fwd", "msa_bwd", "msa_check_status", "msa_diag_umma",
               "msa_diag_wait_timeout", "msa_set_kernel_events"):
         getattr(lib, f).restype = I
@@ -201,6 +203,11 @@ def set_kernel_events(kernel: int, start=None, stop=None) -> None:
     s = ctypes.c_void_p(start.cuda_event) if start is not None else None
     e = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
     _check(LIB.msa_set_kernel_events(kernel, s, e), "msa_set_kernel_events")
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(LIB.msa_kernel_launches())
 
 
 def diag_umma(mode: int, A: torch.Tensor, B: torch.Tensor) -> torch.Tensor:

@@ -168,6 +168,11 @@ enum msa_kernel { MSA_KERNEL_PROXY = 0, MSA_KERNEL_FWD_MAIN = 1, MSA_KERNEL_BWD_
  * NULL stops recording.  The events stay owned by the caller. */
 MSA_API int msa_set_kernel_events(int kernel, void* start, void* stop);
 
+/* Number of kernels this library has enqueued in this process since it was
+ * loaded (every launch of every entry point, counted on the host as it is
+ * made; thread-safe).  Callers take the difference around a region. */
+MSA_API uint64_t msa_kernel_launches(void);
+
 /* ---- diagnostics (no counterpart on the pages; used by the GPU tests) ---- */
 
 /* One 128 x N x K tcgen05 MMA, D[m][n] = sum_k A[m][k] * B[n][k], with the
