@@ -196,7 +196,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&st_empty[s]);   // staging read: the stage may be refilled
         }
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        // the shared-memory source must have been read before the CTA exits;
+        // the global side completes on its own
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
@@ -462,7 +464,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                  : "memory");
                 }
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             }
         }
     }

@@ -302,7 +302,9 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             }
         }
-        if (issued) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        // the staging must have been read before the CTA exits; the global
+        // side completes on its own
+        if (issued) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
 
     __syncthreads();
