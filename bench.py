@@ -133,6 +133,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary of this
+    workload, or None when there is none or the kernel's sources have changed
+    since it was captured (the summary records their sha256)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"dram_msa_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    csrc = os.path.join(ROOT, "block_sparse_attention_09_b200", "csrc")
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 5 and parts[0] == "traffic" and parts[1] == kernel:
+            h = hashlib.sha256()
+            for name in parts[3].split(","):
+                fp = os.path.join(csrc, name)
+                if not os.path.exists(fp):
+                    return None
+                with open(fp, "rb") as f:
+                    h.update(f.read())
+            return float(parts[2]) if h.hexdigest() == parts[4] else None
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -399,7 +422,8 @@ def main():
     achieved = kf[dom] / (kern_ms[dom] * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": None,
+            "frac": achieved / peak, "traffic": recorded_traffic(dom, cfg.name),
+            "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
             "frac_of_burst": achieved / float(peaks.get("bf16_tflops", peak))}
 
