@@ -50,7 +50,8 @@ def build(force: bool = False) -> str:
 class _Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("Hq", ctypes.c_int),
                 ("Hkv", ctypes.c_int), ("d", ctypes.c_int), ("dp", ctypes.c_int),
-                ("blk", ctypes.c_int), ("topk", ctypes.c_int), ("scale", ctypes.c_double)]
+                ("blk", ctypes.c_int), ("topk", ctypes.c_int), ("scale", ctypes.c_double),
+                ("window", ctypes.c_int), ("dilation", ctypes.c_int)]
 
 
 def _load():
@@ -60,7 +61,8 @@ def _load():
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         _lib.msa_oracle_select.argtypes = [ctypes.POINTER(_Dims), P, P, I64, P, P, P, P, ctypes.c_int]
-        _lib.msa_oracle_select_from_pooled.argtypes = [I64, ctypes.c_int, ctypes.c_int, P, P, P, P]
+        _lib.msa_oracle_select_from_pooled.argtypes = [I64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                       P, P, P, P]
         _lib.msa_oracle_fwd.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, I64, P, P, P, ctypes.c_int]
         _lib.msa_oracle_bwd_dq.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, P, P, P, I64, P,
                                            P, P, ctypes.c_int]
@@ -84,6 +86,8 @@ class Dims:
     topk: int
     blk: int = 128
     scale: float = 0.0  # 0 -> 1/sqrt(d)
+    window: int = 1     # forced blocks: own block and the window-1 before it,
+    dilation: int = 1   # every `dilation`-th block
 
     @property
     def nblk(self) -> int:
@@ -95,7 +99,8 @@ class Dims:
 
     def c(self) -> _Dims:
         s = self.scale if self.scale else 1.0 / np.sqrt(self.d)
-        return _Dims(self.B, self.T, self.Hq, self.Hkv, self.d, self.dp, self.blk, self.topk, s)
+        return _Dims(self.B, self.T, self.Hq, self.Hkv, self.d, self.dp, self.blk, self.topk, s,
+                     self.window, self.dilation)
 
 
 def _f32(a):
@@ -138,7 +143,7 @@ def select(m: Dims, qp, kp, rows=None, want_pooled=False, idx=None, nsel=None, n
     return idx, nsel, pooled
 
 
-def select_from_pooled(pooled, bi, topk):
+def select_from_pooled(pooled, bi, topk, window=1, dilation=1):
     """The selection rule alone on given float32 scores [nrows, nblk] with the
     query's own block per row: returns (idx [nrows, topk], nsel [nrows])."""
     lib = _load()
@@ -147,7 +152,8 @@ def select_from_pooled(pooled, bi, topk):
     bi = np.ascontiguousarray(np.asarray(bi, dtype=np.int32))
     idx = np.empty((nrows, topk), dtype=np.int32)
     nsel = np.empty((nrows,), dtype=np.int32)
-    lib.msa_oracle_select_from_pooled(nrows, nb, topk, _ptr(pooled), _ptr(bi), _ptr(idx), _ptr(nsel))
+    lib.msa_oracle_select_from_pooled(nrows, nb, topk, window, dilation, _ptr(pooled), _ptr(bi), _ptr(idx),
+                                      _ptr(nsel))
     return idx, nsel
 
 

@@ -44,6 +44,7 @@
 typedef struct {
     int B, T, Hq, Hkv, d, dp, blk, topk;
     double scale;
+    int window, dilation;   /* forced block pattern; 1, 1: only the own block */
 } odims;
 
 static int nblocks(const odims* m) { return (m->T + m->blk - 1) / m->blk; }
@@ -139,21 +140,43 @@ static int int_cmp(const void* pa, const void* pb)
     return (a > b) - (a < b);
 }
 
-/* Selection for one row: the query's own block bi is always kept; the other
- * topk-1 slots go to the best blocks among 0..bi-1 in the order above.  If
- * the query has at most topk eligible blocks it takes all of them.  Output is
- * ascending and padded with -1; returns the count. */
-static int select_row(const float* pooled, int bi, int topk, int32_t* out, cand* scratch)
+/* Forced blocks of a query in block bi under a window of `window` blocks with
+ * dilation `dilation` (page "Flash-MSA: Train on a million tokens without
+ * breaking the compute bank", section "Under the hood": the block pattern is
+ * configurable by window size and dilation; our reading): bi, bi - dilation,
+ * ..., bi - (window-1) dilation, those that are >= 0.  window = 1 forces only
+ * the own block.  Returns 1 if block n is forced. */
+static int is_forced(int n, int bi, int window, int dilation)
+{
+    const int back = bi - n;
+    return back >= 0 && back % dilation == 0 && back / dilation < window;
+}
+
+/* Selection for one row: the forced blocks (the query's own block bi, plus the
+ * window) are always kept; the remaining slots of the topk go to the best of
+ * the other blocks 0..bi in the order above.  If the query has at most topk
+ * eligible blocks it takes all of them.  Output is ascending and padded with
+ * -1; returns the count. */
+static int select_row(const float* pooled, int bi, int topk, int window, int dilation, int32_t* out,
+                      cand* scratch)
 {
     int cnt = 0;
     int* sel = (int*)out;
     if (bi + 1 <= topk) {
         for (int n = 0; n <= bi; ++n) sel[cnt++] = n;
     } else {
-        for (int n = 0; n < bi; ++n) { scratch[n].s = pooled[n]; scratch[n].n = n; }
-        qsort(scratch, (size_t)bi, sizeof(cand), cand_cmp);
-        for (int r = 0; r < topk - 1; ++r) sel[cnt++] = scratch[r].n;
-        sel[cnt++] = bi;
+        int nc = 0;
+        for (int n = 0; n <= bi; ++n) {
+            if (is_forced(n, bi, window, dilation)) {
+                sel[cnt++] = n;
+            } else {
+                scratch[nc].s = pooled[n];
+                scratch[nc].n = n;
+                ++nc;
+            }
+        }
+        qsort(scratch, (size_t)nc, sizeof(cand), cand_cmp);
+        for (int r = 0; cnt < topk && r < nc; ++r) sel[cnt++] = scratch[r].n;
         qsort(sel, (size_t)cnt, sizeof(int), int_cmp);
     }
     for (int r = cnt; r < topk; ++r) out[r] = -1;
@@ -182,7 +205,7 @@ static void sel_item(void* vctx, int64_t r)
     pool_row(m, c->qp, c->kp, b, g, i, pooled);
     if (c->pooled_out) memcpy(c->pooled_out + r * nb, pooled, sizeof(float) * (size_t)nb);
     int32_t* out = c->idx + row * m->topk;
-    c->nsel[row] = select_row(pooled, i / m->blk, m->topk, out, scratch);
+    c->nsel[row] = select_row(pooled, i / m->blk, m->topk, m->window, m->dilation, out, scratch);
     free(pooled);
     free(scratch);
 }
@@ -199,13 +222,13 @@ int msa_oracle_select(const odims* m, const float* qp, const float* kp,
 
 /* Selection alone, from given pooled rows [nrows][nblk] with the query's
  * block index per row (used to check a selection rule on fixed scores). */
-int msa_oracle_select_from_pooled(int64_t nrows, int nblk, int topk,
+int msa_oracle_select_from_pooled(int64_t nrows, int nblk, int topk, int window, int dilation,
                                   const float* pooled, const int32_t* bi,
                                   int32_t* idx, int32_t* nsel)
 {
     cand* scratch = (cand*)malloc(sizeof(cand) * (size_t)(nblk > 0 ? nblk : 1));
     for (int64_t r = 0; r < nrows; ++r)
-        nsel[r] = select_row(pooled + r * nblk, bi[r], topk, idx + r * topk, scratch);
+        nsel[r] = select_row(pooled + r * nblk, bi[r], topk, window, dilation, idx + r * topk, scratch);
     free(scratch);
     return 0;
 }

@@ -96,6 +96,59 @@ def test_select_golden_cases():
         assert int(nsel[0]) == c["nsel"], c["why"]
 
 
+def test_golden_selection_window_cases():
+    """Hand-derived cases for the forced window / dilation pattern."""
+    with open(os.path.join(HERE, "golden", "select_window_cases.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        pooled = np.array([c["pooled"]], dtype=np.float32)
+        idx, nsel = O.select_from_pooled(pooled, [c["bi"]], c["topk"], c["window"], c["dilation"])
+        assert idx[0].tolist() == c["idx"], c["why"]
+        assert int(nsel[0]) == c["nsel"], c["why"]
+
+
+def test_window_one_is_the_plain_rule():
+    """window 1 forces only the own block: the plain rule, for any dilation."""
+    rng = np.random.default_rng(3)
+    pooled = rng.integers(-3, 4, size=(400, 40)).astype(np.float32)   # many ties
+    bi = rng.integers(0, 40, size=400).astype(np.int32)
+    for topk in (1, 3, 8):
+        a, na = O.select_from_pooled(pooled, bi, topk)
+        for dil in (1, 2, 5):
+            b, nb = O.select_from_pooled(pooled, bi, topk, 1, dil)
+            assert np.array_equal(a, b) and np.array_equal(na, nb)
+
+
+def test_window_selection_invariants():
+    """For any scores: the forced blocks that exist are kept, the count is
+    min(topk, bi+1), and every kept free block ranks above every dropped free
+    block (higher score, or equal score and lower id)."""
+    rng = np.random.default_rng(4)
+    nb = 48
+    pooled = rng.integers(-4, 5, size=(300, nb)).astype(np.float32)
+    bi = rng.integers(0, nb, size=300).astype(np.int32)
+    for topk, window, dil in ((6, 3, 1), (8, 4, 3), (5, 5, 2), (12, 2, 7)):
+        idx, nsel = O.select_from_pooled(pooled, bi, topk, window, dil)
+        for r in range(len(bi)):
+            b_ = int(bi[r])
+            sel = [int(x) for x in idx[r, :nsel[r]]]
+            assert nsel[r] == min(topk, b_ + 1)
+            assert sel == sorted(set(sel)) and all(0 <= x <= b_ for x in sel)
+            assert all(x == -1 for x in idx[r, nsel[r]:])
+            if b_ + 1 <= topk:
+                assert sel == list(range(b_ + 1))
+                continue
+            forced = {b_ - m * dil for m in range(window) if b_ - m * dil >= 0}
+            assert forced <= set(sel)
+            free_kept = [x for x in sel if x not in forced]
+            free_dropped = [x for x in range(b_ + 1) if x not in forced and x not in sel]
+            assert len(free_kept) == topk - len(forced)
+            for k in free_kept:
+                for d_ in free_dropped:
+                    sk, sd = pooled[r, k], pooled[r, d_]
+                    assert sk > sd or (sk == sd and k < d_)
+
+
 def check_selection_invariants(pooled_row, bi, topk, idx_row, nsel):
     sel = [int(x) for x in idx_row[:nsel]]
     assert nsel == min(topk, bi + 1)
@@ -123,6 +176,20 @@ def test_pool_matches_full_score_matrix(oracle_mod, blk, T, topk):
         i = r % m.T
         check_selection_invariants(pooled[r], i // blk, topk, idx.reshape(-1, topk)[r],
                                    int(nsel.reshape(-1)[r]))
+
+
+@pytest.mark.parametrize("window,dil", [(3, 1), (4, 2), (2, 5)])
+def test_select_window_end_to_end(oracle_mod, window, dil):
+    """Proxy scores -> pool -> windowed selection agrees with the rule applied
+    to the numpy-pooled full score matrix (the pooling pin above)."""
+    m = Dims(B=1, T=1280, Hq=2, Hkv=2, d=16, dp=32, topk=6, blk=128, window=window, dilation=dil)
+    x = rand_inputs(m, seed=window * 10 + dil, grid=True)
+    idx, nsel, _ = O.select(m, x["qp"], x["kp"])
+    ref = bf_pooled(m, x["qp"], x["kp"]).reshape(-1, m.nblk)
+    bi = (np.arange(ref.shape[0]) % m.T) // m.blk
+    ridx, rnsel = O.select_from_pooled(ref, bi, m.topk, window, dil)
+    assert np.array_equal(idx.reshape(-1, m.topk), ridx)
+    assert np.array_equal(nsel.reshape(-1), rnsel)
 
 
 def test_pool_float_inputs_close(oracle_mod):
