@@ -41,15 +41,18 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="query rows in the CPU sample (0 = auto)")
+    ap.add_argument("--window", type=int, default=1, help="forced blocks per query (own block included)")
+    ap.add_argument("--dilation", type=int, default=1, help="stride between forced blocks")
     ap.add_argument("--bias", default=None, choices=["none", "group", "recency"],
                     help="override the workload's proxy-input structure (profiling variants)")
     return ap.parse_args()
 
 
-def workload_name(cfg):
+def workload_name(cfg, window=1, dilation=1):
     bias = {"none": "", "group": ", per-group low-rank proxy bias", "recency": ", planted local-recency proxy bias"}
+    pattern = f", forced window {window} blocks at dilation {dilation}" if window > 1 else ""
     return (f"MSA {cfg.name}: B={cfg.B} T={cfg.T} Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} dp={cfg.dp} "
-            f"topk={cfg.topk} (own block incl.), causal, fwd+bwd{bias[cfg.bias]}")
+            f"topk={cfg.topk} (own block incl.), causal, fwd+bwd{bias[cfg.bias]}{pattern}")
 
 
 # ---------------------------------------------------------------- FLOP model
@@ -186,14 +189,15 @@ def oracle_arrays(host):
     return {k: v.float().numpy() for k, v in host.items()}
 
 
-def cpu_oracle_sample(cfg, x, rows_target, seed=0):
+def cpu_oracle_sample(cfg, x, rows_target, seed=0, window=1, dilation=1):
     """Time the oracle on a bounded sample of query rows (b, g, i) of the
     workload: selection (proxy scores of the row over all earlier keys, pool,
     top-k), then forward, dQ and the row's dK/dV contributions for each of
     the group's G heads.  Returns (credited FLOPs, seconds, rows, threads)."""
     import oracle as O
     from block_sparse_attention_09_b200.inputs import sample_rows
-    m = O.Dims(B=cfg.B, T=cfg.T, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, dp=cfg.dp, topk=cfg.topk)
+    m = O.Dims(B=cfg.B, T=cfg.T, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, dp=cfg.dp, topk=cfg.topk, window=window,
+               dilation=dilation)
     threads = os.cpu_count() or 1
     srows = sample_rows(cfg.B * cfg.Hkv * cfg.T, rows_target, seed=seed + 11)
     t0 = time.perf_counter()
@@ -225,9 +229,9 @@ def cpu_oracle_sample(cfg, x, rows_target, seed=0):
     return flops, secs, len(srows), threads
 
 
-def calibrate_rows(cfg, x, seconds, cap=4096):
+def calibrate_rows(cfg, x, seconds, cap=4096, window=1, dilation=1):
     """Rows of the CPU sample that take about `seconds` on this host."""
-    fl, secs, n, _ = cpu_oracle_sample(cfg, x, 32, seed=99)
+    fl, secs, n, _ = cpu_oracle_sample(cfg, x, 32, seed=99, window=window, dilation=dilation)
     return max(8, min(cap, int(n * seconds / max(secs, 1e-3))))
 
 
@@ -236,10 +240,10 @@ def run_reference(args, cfg, rank):
         return
     from block_sparse_attention_09_b200.inputs import make_inputs
     x = oracle_arrays(make_inputs(cfg, seed=0))
-    rows = args.cpu_rows or calibrate_rows(cfg, x, seconds=4.0)
+    rows = args.cpu_rows or calibrate_rows(cfg, x, seconds=4.0, window=args.window, dilation=args.dilation)
     vals = []
     for s in range(args.warmup + args.steps):
-        fl, secs, n, threads = cpu_oracle_sample(cfg, x, rows, seed=s)
+        fl, secs, n, threads = cpu_oracle_sample(cfg, x, rows, seed=s, window=args.window, dilation=args.dilation)
         if s >= args.warmup:
             vals.append((fl, secs))
     fl = sum(v[0] for v in vals)
@@ -249,7 +253,7 @@ def run_reference(args, cfg, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(vals),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": workload_name(cfg)},
+            "data": "synthetic", "config": {"workload": workload_name(cfg, args.window, args.dilation)},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -298,7 +302,8 @@ def main():
     def step(inputs, ev=None):
         if ev is not None:
             ev[0].record(stream)
-        idx, nsel = msa.proxy_select(inputs["qp"], inputs["kp"], cfg.topk, ws=ws_sel)
+        idx, nsel = msa.proxy_select(inputs["qp"], inputs["kp"], cfg.topk, ws=ws_sel, window=args.window,
+                                     dilation=args.dilation)
         if ev is not None:
             ev[1].record(stream)
         msa.fwd(inputs["q"], inputs["k"], inputs["v"], idx, nsel, ws=ws_fwd, out=(o, lse))
@@ -430,8 +435,8 @@ def main():
     cpu = None
     if not args.no_cpu and world == 1:
         x = oracle_arrays(host)
-        rows = args.cpu_rows or calibrate_rows(cfg, x, seconds=15.0)
-        fl, secs, n, threads = cpu_oracle_sample(cfg, x, rows, seed=0)
+        rows = args.cpu_rows or calibrate_rows(cfg, x, seconds=15.0, window=args.window, dilation=args.dilation)
+        fl, secs, n, threads = cpu_oracle_sample(cfg, x, rows, seed=0, window=args.window, dilation=args.dilation)
         cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} query rows (b, group, i) of the same workload, all {cfg.G} heads each: "
                          f"selection, forward, dQ and dK/dV contributions; {secs:.1f} s"}
@@ -441,7 +446,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) bf16 inputs" + (", planted local-recency proxy bias" if cfg.bias == "recency" else ""),
-        "config": {"workload": workload_name(cfg), "B": B, "T": T, "Hq": Hq, "Hkv": Hkv, "d": D,
+        "config": {"workload": workload_name(cfg, args.window, args.dilation), "B": B, "T": T, "Hq": Hq, "Hkv": Hkv, "d": D,
                    "dp": cfg.dp, "topk": cfg.topk, "per_rank": "one batch per rank (seed = rank)",
                    "l2": "inputs larger than L2 (Q alone %.2f GB), no flush" % (d["q"].numel() * 2 / 1e9)},
         "tokens_per_s": tok_s,

@@ -106,9 +106,12 @@ int to_problem(const msa_dims* d, Problem* p)
     if (d->d != 64 && d->d != 128) return MSA_ERR_INVALID_DIMS;
     if (d->dp < 8 || d->dp > 64 || d->dp % 8 != 0) return MSA_ERR_INVALID_DIMS;
     if (!isfinite(d->scale)) return MSA_ERR_INVALID_DIMS;
+    if (d->window < 0 || d->window > d->topk || d->dilation < 0 || d->dilation > kMaxT) return MSA_ERR_INVALID_DIMS;
     p->B = d->B; p->T = d->T; p->Hq = d->Hq; p->Hkv = d->Hkv; p->Hp = d->Hp;
     p->d = d->d; p->dp = d->dp; p->topk = d->topk;
     p->nblk = (d->T + kBlock - 1) / kBlock;
+    p->window = d->window > 0 ? d->window : 1;
+    p->dilation = d->dilation > 0 ? d->dilation : 1;
     p->G = G;
     p->scale = d->scale != 0.f ? d->scale : 1.0f / sqrtf((float)d->d);
     if ((int64_t)p->B * p->Hp * p->T * p->topk > (int64_t)INT32_MAX) return MSA_ERR_INVALID_DIMS;

@@ -23,6 +23,7 @@ enum KernelId : uint32_t { kKidProxy = 1, kKidFwd = 2, kKidBwd = 3, kKidDiag = 4
 
 struct Problem {
     int B, T, Hq, Hkv, Hp, d, dp, topk, nblk, G;
+    int window, dilation;   // forced block pattern of the selection (>= 1)
     float scale;
     int64_t rows_q() const { return (int64_t)B * T * Hq; }
 };

@@ -45,6 +45,7 @@ constexpr int kPend = 10;                  // pending slots per row (merge once 
 
 struct Params {
     int B, T, Hp, dp, nblk, topk;
+    int window, dilation;   // forced blocks: qb, qb - dilation, ... (window of them)
     int32_t* idx;
     int32_t* nsel;
     float* pooled;     // optional
@@ -121,9 +122,10 @@ MSA_DEV void warp_sort(int (&v)[V])
 }
 
 // The warp's 32 rows (TMEM lane quarter q): ascending output of each row's
-// kept ids plus the own block, -1 padded; one row at a time, V ids per lane.
+// k1 kept ids and the topk - k1 forced blocks qb, qb - dil, ...; one row at a
+// time, V ids per lane.
 template <int V>
-MSA_DEV void write_selection(const uint2* heap, int k1, int topk, int q, int qb, int T, int64_t row0,
+MSA_DEV void write_selection(const uint2* heap, int k1, int topk, int dil, int q, int qb, int T, int64_t row0,
                              int32_t* idx, int32_t* nsel)
 {
     const int lane = (int)(threadIdx.x & 31u);
@@ -133,7 +135,8 @@ MSA_DEV void write_selection(const uint2* heap, int k1, int topk, int q, int qb,
 #pragma unroll
         for (int w = 0; w < V; ++w) {
             const int slot = V * lane + w;
-            v[w] = slot < k1 ? (int)heap[slot * 128 + row].y : 0x7fffffff;
+            v[w] = slot < k1 ? (int)heap[slot * 128 + row].y
+                             : (slot < topk ? qb - (slot - k1) * dil : 0x7fffffff);
         }
         warp_sort<V>(v);
         const int i = qb * 128 + row;
@@ -142,18 +145,32 @@ MSA_DEV void write_selection(const uint2* heap, int k1, int topk, int q, int qb,
 #pragma unroll
             for (int w = 0; w < V; ++w) {
                 const int slot = V * lane + w;
-                if (slot < k1) out[slot] = v[w];
-                else if (slot == k1) out[slot] = qb;
-                else if (slot < topk) out[slot] = -1;
+                if (slot < topk) out[slot] = v[w];
             }
-            if (lane == 0) nsel[row0 + row] = k1 + 1;
+            if (lane == 0) nsel[row0 + row] = topk;
         }
     }
 }
 
+// Output of a row that ranks nothing: every eligible block (take_all), or the
+// nf forced blocks qb - (nf-1) dil, ..., qb.
+MSA_DEV void write_unranked(int32_t* out, int32_t* nsel_out, bool take_all, int qb, int nf, int dil, int topk)
+{
+    int c = 0;
+    if (take_all) {
+        for (int n = 0; n <= qb; ++n) out[c++] = n;
+    } else {
+        for (int m = nf - 1; m >= 0; --m) out[c++] = qb - m * dil;
+    }
+    *nsel_out = c;
+    for (int s = c; s < topk; ++s) out[s] = -1;
+}
+
 // NSTAGE stages of 256 proxy keys (two key blocks) each; two TMEM
-// accumulators of 256 columns (all of TMEM: one CTA per SM).
-template <int NSTAGE>
+// accumulators of 256 columns (all of TMEM: one CTA per SM).  WINDOW: a forced
+// pattern beyond the own block is in use (a separate instance keeps the
+// plain selection's inner loop unchanged).
+template <int NSTAGE, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1)
 proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_kp,
                     Params p)
@@ -168,7 +185,8 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     const int bg = (int)(blockIdx.x / p.nblk);
     const int qb = p.nblk - 1 - (int)(blockIdx.x % p.nblk);
     const int b = bg / p.Hp, g = bg % p.Hp;
-    const int k1 = p.topk - 1;                             // slots besides the own block
+    const int nf = WINDOW ? min(p.window, qb / p.dilation + 1) : 1;   // forced blocks that exist
+    const int k1 = p.topk - nf;                            // slots ranked by pooled score
     const bool dbg = p.pooled != nullptr;
     const bool take_all = qb + 1 <= p.topk;                // every eligible block kept
     const bool need_heap = !take_all && k1 > 0;
@@ -203,18 +221,10 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     const uint32_t code0 = kStTimeoutBase + kKidProxy * 16;
 
     if (ntiles == 0) {
-        // Nothing to rank: the query keeps blocks 0..qb (or only qb when topk == 1).
-        if (row_ok) {
-            int32_t* out = p.idx + ((int64_t)bg * p.T + i) * p.topk;
-            int c = 0;
-            if (take_all) {
-                for (int n = 0; n <= qb; ++n) out[c++] = n;
-            } else {
-                out[c++] = qb;
-            }
-            p.nsel[(int64_t)bg * p.T + i] = c;
-            for (int s = c; s < p.topk; ++s) out[s] = -1;
-        }
+        // Nothing to rank: every eligible block, or only the forced ones.
+        if (row_ok)
+            write_unranked(p.idx + ((int64_t)bg * p.T + i) * p.topk, p.nsel + (int64_t)bg * p.T + i, take_all, qb,
+                           nf, p.dilation, p.topk);
         return;
     }
 
@@ -320,9 +330,16 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
             }
             return fmaxf(fmax3(m0, m1, m2), m3);
         };
+        // blocks arrive in descending order: the next forced block below the own
+        // one is a running pointer (-1 once all nf - 1 of them have passed)
+        int next_forced = nf > 1 ? qb - p.dilation : -1, forced_left = nf - 1;
         auto consume = [&](int n, float mx) {
             if (dbg && row_ok) p.pooled[((int64_t)bg * p.T + i) * p.nblk + n] = mx;
             if (!need_heap || n == qb) return;
+            if (WINDOW && n == next_forced) {   // forced: kept without ranking
+                next_forced = --forced_left > 0 ? n - p.dilation : -1;
+                return;
+            }
             if (cnt < k1) {   // same count for every row of the tile: warp-uniform
                 heap[cnt * 128 + r] = cand(mx, n);
                 if (++cnt == k1) {
@@ -378,19 +395,12 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
             if (need_heap) {
                 const int64_t row0 = (int64_t)bg * p.T + qb * 128;
                 if (p.topk <= 64)
-                    write_selection<2>(heap, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+                    write_selection<2>(heap, k1, p.topk, p.dilation, warp & 3, qb, p.T, row0, p.idx, p.nsel);
                 else
-                    write_selection<4>(heap, k1, p.topk, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+                    write_selection<4>(heap, k1, p.topk, p.dilation, warp & 3, qb, p.T, row0, p.idx, p.nsel);
             } else if (row_ok) {
-                int32_t* out = p.idx + ((int64_t)bg * p.T + i) * p.topk;
-                int c = 0;
-                if (take_all) {
-                    for (int n = 0; n <= qb; ++n) out[c++] = n;
-                } else {
-                    out[c++] = qb;
-                }
-                p.nsel[(int64_t)bg * p.T + i] = c;
-                for (int s = c; s < p.topk; ++s) out[s] = -1;
+                write_unranked(p.idx + ((int64_t)bg * p.T + i) * p.topk, p.nsel + (int64_t)bg * p.T + i, take_all,
+                               qb, nf, p.dilation, p.topk);
             }
             if (dbg && row_ok)
                 for (int n = qb + 1; n < p.nblk; ++n)
@@ -405,11 +415,11 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     }
 }
 
-template <int NSTAGE>
+template <int NSTAGE, bool WINDOW>
 cudaError_t launch_variant(const Problem& pr, const CUtensorMap& tm_qp, const CUtensorMap& tm_kp,
                            const Params& p, size_t smem, cudaStream_t st)
 {
-    auto kern = proxy_select_kernel<NSTAGE>;
+    auto kern = proxy_select_kernel<NSTAGE, WINDOW>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(pr.nblk * pr.B * pr.Hp);
@@ -433,12 +443,19 @@ cudaError_t launch_proxy_select(const Problem& pr, const CUtensorMap& tm_qp, con
                                 int32_t* idx, int32_t* nsel, float* pooled, uint32_t* status,
                                 cudaStream_t st)
 {
-    Params p{pr.B, pr.T, pr.Hp, pr.dp, pr.nblk, pr.topk, idx, nsel, pooled, status};
+    Params p{pr.B, pr.T, pr.Hp, pr.dp, pr.nblk, pr.topk, pr.window, pr.dilation, idx, nsel, pooled, status};
     // All of TMEM per CTA: at least 120 KB of shared memory keeps one CTA per SM.
+    const bool win = pr.window > 1;
     const size_t s4 = smem_bytes(4, pr.topk);
-    if (s4 <= 227 * 1024) return launch_variant<4>(pr, tm_qp, tm_kp, p, s4 < 120 * 1024 ? 120 * 1024 : s4, st);
+    if (s4 <= 227 * 1024) {
+        const size_t sm = s4 < 120 * 1024 ? 120 * 1024 : s4;
+        return win ? launch_variant<4, true>(pr, tm_qp, tm_kp, p, sm, st)
+                   : launch_variant<4, false>(pr, tm_qp, tm_kp, p, sm, st);
+    }
     const size_t s2 = smem_bytes(2, pr.topk);
-    return launch_variant<2>(pr, tm_qp, tm_kp, p, s2 < 120 * 1024 ? 120 * 1024 : s2, st);
+    const size_t sm = s2 < 120 * 1024 ? 120 * 1024 : s2;
+    return win ? launch_variant<2, true>(pr, tm_qp, tm_kp, p, sm, st)
+               : launch_variant<2, false>(pr, tm_qp, tm_kp, p, sm, st);
 }
 
 }  // namespace msa

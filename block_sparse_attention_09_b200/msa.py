@@ -40,7 +40,8 @@ class MsaError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
                 ("Hp", ctypes.c_int), ("d", ctypes.c_int), ("dp", ctypes.c_int), ("block", ctypes.c_int),
-                ("topk", ctypes.c_int), ("scale", ctypes.c_float)]
+                ("topk", ctypes.c_int), ("scale", ctypes.c_float), ("window", ctypes.c_int),
+                ("dilation", ctypes.c_int)]
 
 
 def _load():
@@ -71,8 +72,9 @@ def _load():
 LIB = _load()
 
 
-def make_dims(B, T, Hq, Hkv, d, dp, topk, scale=0.0) -> Dims:
-    return Dims(int(B), int(T), int(Hq), int(Hkv), int(Hkv), int(d), int(dp), 128, int(topk), float(scale))
+def make_dims(B, T, Hq, Hkv, d, dp, topk, scale=0.0, window=1, dilation=1) -> Dims:
+    return Dims(int(B), int(T), int(Hq), int(Hkv), int(Hkv), int(d), int(dp), 128, int(topk), float(scale),
+                int(window), int(dilation))
 
 
 def _p(t):
@@ -117,11 +119,13 @@ def dims_of(q, k, qp, topk, scale=0.0) -> Dims:
     return make_dims(B, T, Hq, Hkv, d, dp, topk, scale)
 
 
-def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False):
-    """Index Branch.  Returns (idx, nsel) or (idx, nsel, pooled_scores)."""
+def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False, window=1, dilation=1):
+    """Index Branch.  Returns (idx, nsel) or (idx, nsel, pooled_scores).
+    window/dilation: forced block pattern (own block and the window-1 blocks
+    every `dilation` blocks before it)."""
     _bf16(qp, kp)
     B, T, Hp, dp = qp.shape
-    dims = make_dims(B, T, Hp, Hp, 64, dp, topk)
+    dims = make_dims(B, T, Hp, Hp, 64, dp, topk, window=window, dilation=dilation)
     idx = torch.empty((B, Hp, T, topk), dtype=torch.int32, device=qp.device)
     nsel = torch.empty((B, Hp, T), dtype=torch.int32, device=qp.device)
     nblk = (T + 127) // 128

@@ -60,6 +60,8 @@ typedef struct msa_dims {
     int block;  /* KV block length: must be 128                           */
     int topk;   /* blocks read per query, own block included              */
     float scale;/* softmax scale of the Main Branch; 0 -> 1/sqrt(d)       */
+    int window; /* forced blocks per query (own block included); 0 -> 1  */
+    int dilation;/* stride between forced blocks; 0 -> 1                 */
 } msa_dims;
 
 enum msa_status {
@@ -88,7 +90,15 @@ MSA_API size_t msa_workspace_size(const msa_dims* dims, int which);
  *   pooled(b,g,i,n) = max of score over the keys of block n (n <= i/128)
  * Query i keeps its own block i/128 and the topk-1 best earlier blocks by
  * pooled score, equal scores going to the lower block id; with at most topk
- * eligible blocks it keeps them all.  idx rows are written ascending and
+ * eligible blocks it keeps them all.
+ *   Forced pattern ("Flash-MSA: Train on a million tokens without breaking
+ *   the compute bank", section "Under the hood": the block pattern is
+ *   configurable by window size and dilation): with window w and dilation s,
+ *   the blocks i/128, i/128 - s, ..., i/128 - (w-1)s that exist are always
+ *   kept and count toward topk; the remaining slots go to the best of the
+ *   other blocks.  w = 1 (the default) forces the own block only.  Requires
+ *   w <= topk.  msa_fwd and msa_bwd read any valid idx and ignore both
+ *   fields.  idx rows are written ascending and
  * padded with -1; nsel = number of valid entries.  Scores are accumulated in
  * fp32 on the tensor cores and compared in fp32; the T x T score matrix
  * never leaves the chip.

@@ -55,6 +55,12 @@ def dims(lib, **kw):
     return lib.make_dims(**base)
 
 
+def test_window_fields_accepted(lib):
+    """window 0..topk and any dilation >= 0 are valid; 0 means 1."""
+    for w, s in ((0, 0), (1, 1), (4, 1), (3, 9), (2, 0)):
+        assert lib.workspace_size(dims(lib, window=w, dilation=s), lib.MSA_SELECT) == 256
+
+
 def test_workspace_sizes(lib):
     d = dims(lib)
     sel = lib.workspace_size(d, lib.MSA_SELECT)
@@ -69,7 +75,8 @@ def test_workspace_sizes(lib):
 
 
 @pytest.mark.parametrize("bad", [dict(d=96), dict(dp=12), dict(dp=72), dict(topk=0), dict(topk=129),
-                                 dict(Hq=6, Hkv=4), dict(Hq=12, Hkv=4), dict(T=-1), dict(T=(1 << 20) + 1)])
+                                 dict(Hq=6, Hkv=4), dict(Hq=12, Hkv=4), dict(T=-1), dict(T=(1 << 20) + 1),
+                                 dict(window=5), dict(window=-1), dict(dilation=-2)])
 def test_invalid_dims_rejected(lib, bad):
     d = dims(lib, **bad)
     assert lib.workspace_size(d, lib.MSA_FWD) == 0
