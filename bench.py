@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="query rows in the CPU sample (0 = auto)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time msa_decode (one new token per sequence against full-length caches) instead")
+    ap.add_argument("--decode-batch", type=int, default=16, help="sequences per decode step")
     ap.add_argument("--window", type=int, default=1, help="forced blocks per query (own block included)")
     ap.add_argument("--dilation", type=int, default=1, help="stride between forced blocks")
     ap.add_argument("--bias", default=None, choices=["none", "group", "recency"],
@@ -260,6 +263,67 @@ def run_reference(args, cfg, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- decode arm
+def run_decode(args, cfg, rank, local):
+    """Decode step: every sequence of the batch attends with one new token to
+    caches of the workload's full length T.  Caches are seeded N(0,1) bf16
+    drawn on the device (the timing does not depend on their values).  Metric:
+    tokens/s; roofline: the HBM bytes a step must read (the proxy-key scan and
+    the selected K/V tiles) over the decode kernels' time."""
+    import torch
+    from block_sparse_attention_09_b200 import msa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, T, Hq, Hkv, D, dp, k = args.decode_batch, cfg.T, cfg.Hq, cfg.Hkv, cfg.d, cfg.dp, cfg.topk
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    mk = lambda *shape: torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    kc, vc, kpc = mk(B, T, Hkv, D), mk(B, T, Hkv, D), mk(B, T, Hkv, dp)
+    q, qp = mk(B, Hq, D), mk(B, Hkv, dp)
+    dims = msa.make_dims(B, T, Hq, Hkv, D, dp, k, window=args.window, dilation=args.dilation)
+    ws = msa.workspace(dims, msa.MSA_DECODE, dev)
+    out = (torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev), torch.empty((B, Hq), dtype=torch.float32, device=dev),
+           torch.empty((B, Hkv, k), dtype=torch.int32, device=dev), torch.empty((B, Hkv), dtype=torch.int32, device=dev))
+    step = lambda: msa.decode(q, qp, kc, vc, kpc, k, ws=ws, out=out, window=args.window, dilation=args.dilation)
+    step()
+    if msa.check_status(ws) != 0:
+        raise RuntimeError("device status on the decode workload")
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(args.steps, 20)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = msa.kernel_launches()
+    a.record()
+    for _ in range(steps):
+        step()
+    b_.record()
+    torch.cuda.synchronize()
+    launches = msa.kernel_launches() - l0
+    ms = a.elapsed_time(b_) / steps
+    # bytes a step must read: the proxy keys of every position, and the selected K and V rows
+    nb = (T + 127) // 128
+    rows_sel = min(k, nb) * 128
+    bytes_step = B * Hkv * (T * dp * 2 + 2 * rows_sel * D * 2)
+    peaks, src = measured_peaks()
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    line = {"metric": "MSA decode tokens/s (one new token per sequence, full-length caches)",
+            "value": B / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) bf16 caches drawn on the device",
+            "config": {"workload": (f"MSA decode: {B} sequences x 1 new token, caches T={T} Hq={Hq} Hkv={Hkv} d={D} "
+                                    f"dp={dp} topk={k} (own block incl.)"
+                                    + (f", forced window {args.window} at dilation {args.dilation}"
+                                       if args.window > 1 else "")),
+                       "batch": B, "T": T, "Hq": Hq, "Hkv": Hkv, "d": D, "dp": dp, "topk": k,
+                       "l2": "caches larger than L2 (proxy keys alone %.2f GB), no flush" % (B * T * Hkv * dp * 2 / 1e9)},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                         "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
+                         "algorithmic_bytes_per_step": bytes_step, "peak_source": src},
+            "gpu_launches": launches}
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     args = parse()
@@ -273,6 +337,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, cfg, rank)
+        return
+    if args.decode:
+        run_decode(args, cfg, rank, local)
         return
 
     import torch

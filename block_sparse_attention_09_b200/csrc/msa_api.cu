@@ -34,6 +34,10 @@ WsLayout ws_layout(const Problem& p, int which)
         L.nflag = take(4);
         L.flags = take(rows * 4);
     }
+    if (which == MSA_DECODE) {
+        L.pooled = take(BH * p.nblk * 4);
+        L.part = take((size_t)p.B * p.Hkv * decode_splits(p) * p.G * (p.d + 2) * 4);
+    }
     if (which == MSA_BWD) {
         L.dsum = take(rows * 4);
         L.dqacc = take(rows * p.d * 4);
@@ -95,7 +99,9 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
-int to_problem(const msa_dims* d, Problem* p)
+// decode: idx holds one row per (b, group), so the full-sequence index bound
+// does not apply
+int to_problem(const msa_dims* d, Problem* p, bool decode = false)
 {
     if (!d) return MSA_ERR_NULL_PTR;
     if (d->B < 0 || d->T < 0 || d->T > kMaxT || d->Hkv < 1 || d->Hq < 1 || d->Hq % d->Hkv != 0 ||
@@ -114,7 +120,7 @@ int to_problem(const msa_dims* d, Problem* p)
     p->dilation = d->dilation > 0 ? d->dilation : 1;
     p->G = G;
     p->scale = d->scale != 0.f ? d->scale : 1.0f / sqrtf((float)d->d);
-    if ((int64_t)p->B * p->Hp * p->T * p->topk > (int64_t)INT32_MAX) return MSA_ERR_INVALID_DIMS;
+    if (!decode && (int64_t)p->B * p->Hp * p->T * p->topk > (int64_t)INT32_MAX) return MSA_ERR_INVALID_DIMS;
     return MSA_OK;
 }
 
@@ -144,8 +150,8 @@ extern "C" {
 size_t msa_workspace_size(const msa_dims* dims, int which)
 {
     Problem p;
-    if (to_problem(dims, &p) != MSA_OK) return 0;
-    if (which < MSA_SELECT || which > MSA_BWD) return 0;
+    if (to_problem(dims, &p, which == MSA_DECODE) != MSA_OK) return 0;
+    if (which < MSA_SELECT || which > MSA_DECODE) return 0;
     return ws_layout(p, which).total;
 }
 
@@ -226,6 +232,28 @@ int msa_bwd(const msa_dims* dims, const void* q, const void* k, const void* v, c
     if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     if (launch_block_index(p, idx, nsel, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     if (launch_bwd(p, q, dout, tk, tv, o, lse, dq, dk, dv, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    return MSA_OK;
+}
+
+int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q, const void* qp, const void* k,
+               const void* v, const void* kp, int32_t* idx, int32_t* nsel, void* o, float* lse, void* ws,
+               size_t ws_bytes, void* stream)
+{
+    Problem p;
+    int rc = to_problem(dims, &p, true);
+    if (rc != MSA_OK) return rc;
+    WsLayout L;
+    if ((rc = check_ws(p, MSA_DECODE, ws, ws_bytes, &L)) != MSA_OK) return rc;
+    if (empty(p)) return MSA_OK;
+    if (!q || !qp || !k || !v || !kp || !idx || !nsel || !o || !lse) return MSA_ERR_NULL_PTR;
+    if (!aligned(q, 16) || !aligned(qp, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(kp, 16) ||
+        !aligned(idx, 4) || !aligned(nsel, 4) || !aligned(o, 16) || !aligned(lse, 4) || (lens && !aligned(lens, 4)))
+        return MSA_ERR_MISALIGNED;
+    if ((rc = check_device()) != MSA_OK) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t* status = (uint32_t*)((uint8_t*)ws + L.status);
+    if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    if (launch_decode(p, lens, q, qp, k, v, kp, idx, nsel, o, lse, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     return MSA_OK;
 }
 

@@ -34,6 +34,7 @@ struct WsLayout {
     size_t cnt = 0, tot = 0, ptr = 0, tok = 0;   // block -> query inverse index
     size_t qnorm = 0, kmax = 0, oacc = 0, lacc = 0, nflag = 0, flags = 0;   // forward
     size_t dsum = 0, dqacc = 0, dkacc = 0, dvacc = 0;   // backward
+    size_t pooled = 0, part = 0;                        // decode
     size_t total = 0;
 };
 WsLayout ws_layout(const Problem& p, int which);
@@ -62,6 +63,13 @@ struct TraceEvents {
     cudaEvent_t stop[kTraceCount] = {nullptr, nullptr, nullptr};
 };
 TraceEvents& trace_events();   // per host thread
+// Decode: splits of a row's selected blocks (one attention CTA each) and the
+// launch of the four decode kernels.
+int decode_splits(const Problem& p);
+cudaError_t launch_decode(const Problem& pr, const int32_t* lens, const void* q, const void* qp, const void* k,
+                          const void* v, const void* kp, int32_t* idx, int32_t* nsel, void* o, float* lse,
+                          void* ws, const WsLayout& L, cudaStream_t st);
+
 // Host-side count of kernel launches (msa_kernel_launches).
 void count_launches(unsigned n);
 

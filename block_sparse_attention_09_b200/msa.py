@@ -24,7 +24,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
-MSA_SELECT, MSA_FWD, MSA_BWD = 0, 1, 2
+MSA_SELECT, MSA_FWD, MSA_BWD, MSA_DECODE = 0, 1, 2, 3
 _ERR = {0: "ok", -1: "invalid dimensions", -2: "null pointer", -3: "misaligned pointer",
         -4: "workspace too small", -5: "CUDA launch failed", -6: "device wait timed out",
         -7: "device is not sm_100", -8: "tensor map encoding failed",
@@ -61,6 +61,8 @@ def _load():
     lib.msa_diag_umma.argtypes = [I, I, I, P, P, P, P, P]
     lib.msa_diag_wait_timeout.argtypes = [U64, P, P]
     lib.msa_set_kernel_events.argtypes = [I, P, P]
+    lib.msa_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    lib.msa_decode.restype = I
     lib.msa_kernel_launches.argtypes = []
     lib.msa_kernel_launches.restype = U64
     for f in ("msa_proxy_select", "msa_fwd", "msa_bwd", "msa_check_status", "msa_diag_umma",
@@ -207,6 +209,34 @@ def set_kernel_events(kernel: int, start=None, stop=None) -> None:
     s = ctypes.c_void_p(start.cuda_event) if start is not None else None
     e = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
     _check(LIB.msa_set_kernel_events(kernel, s, e), "msa_set_kernel_events")
+
+
+def decode(q, qp, k, v, kp, topk, lens=None, scale=0.0, window=1, dilation=1, stream=None, ws=None,
+           check=False, out=None):
+    """One new token per sequence against caches.  q [B,Hq,d], qp [B,Hp,dp],
+    caches k, v [B,T,Hkv,d], kp [B,T,Hp,dp]; lens int32 [B] on the device (None:
+    every sequence has length T).  Returns (o [B,Hq,d] bf16, lse [B,Hq] fp32,
+    idx [B,Hp,topk], nsel [B,Hp])."""
+    _bf16(q, qp, k, v, kp)
+    B, T, Hkv, d = k.shape
+    Hq, Hp, dp = q.shape[1], kp.shape[2], kp.shape[3]
+    dims = make_dims(B, T, Hq, Hkv, d, dp, topk, scale, window, dilation)
+    if out is None:
+        o = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        idx = torch.empty((B, Hp, topk), dtype=torch.int32, device=q.device)
+        nsel = torch.empty((B, Hp), dtype=torch.int32, device=q.device)
+    else:
+        o, lse, idx, nsel = out
+    if lens is not None:
+        assert lens.dtype == torch.int32 and lens.is_cuda and lens.is_contiguous()
+    if ws is None:
+        ws = workspace(dims, MSA_DECODE, q.device)
+    _check(LIB.msa_decode(ctypes.byref(dims), _p(lens), _p(q), _p(qp), _p(k), _p(v), _p(kp), _p(idx), _p(nsel),
+                          _p(o), _p(lse), _p(ws), ws.numel(), _stream(stream)), "msa_decode")
+    if check:
+        _check(check_status(ws, stream), "msa_decode (device)")
+    return o, lse, idx, nsel
 
 
 def kernel_launches() -> int:

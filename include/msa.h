@@ -77,7 +77,7 @@ enum msa_status {
     MSA_ERR_INDEX = -9          /* an idx entry outside its valid range       */
 };
 
-enum msa_phase { MSA_SELECT = 0, MSA_FWD = 1, MSA_BWD = 2 };
+enum msa_phase { MSA_SELECT = 0, MSA_FWD = 1, MSA_BWD = 2, MSA_DECODE = 3 };
 
 /* Bytes of workspace `which` (an msa_phase) needs for these dims.
  * Returns 0 for invalid dims. */
@@ -159,6 +159,32 @@ MSA_API int msa_bwd(const msa_dims* dims, const void* q, const void* k, const vo
  */
 MSA_API int msa_fwd_noalloc(const msa_dims* dims, const void* q, const void* k, const void* v,
                             const int32_t* idx, const int32_t* nsel, void* o, float* lse, void* stream);
+
+/*
+ * Decode: attention of one new query token per sequence against caches, with
+ * its own block selection (the inference side of the Index and Main
+ * Branches: "How MSA works"; the MiniMax inference kernels are not public, so
+ * this is our construction from the same two steps).  For sequence b the
+ * token sits at position i = lens[b] - 1 (lens NULL: every sequence has
+ * length T); its key, value and proxy key must already be in the caches.
+ * Computes exactly what msa_proxy_select + msa_fwd compute for the last row
+ * of a sequence of length lens[b]: the pooled proxy scores of i against keys
+ * 0..i, the selection (own block, forced window, topk - nf best others; same
+ * order and ties), then softmax attention of the G heads over the selected
+ * keys j <= i.
+ *   q   [B][Hq][d] bf16, qp [B][Hp][dp] bf16   (the new token)
+ *   k, v [B][T][Hkv][d] bf16, kp [B][T][Hp][dp] bf16   (caches, T = capacity)
+ *   lens [B] int32 on the device, 1 <= lens[b] <= T (others: status word set,
+ *        the sequence gets nsel 0, O = 0 and lse = -inf)
+ *   idx [B][Hp][topk] int32 out (ascending, -1 padded), nsel [B][Hp] out
+ *   o [B][Hq][d] bf16 out, lse [B][Hq] fp32 out (natural log)
+ *   ws: msa_workspace_size(dims, MSA_DECODE) bytes.
+ * Scores are accumulated in fp32 on CUDA cores (the work per token is a few
+ * MFLOP; the cache reads set the time).
+ */
+MSA_API int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q, const void* qp, const void* k,
+                       const void* v, const void* kp, int32_t* idx, int32_t* nsel, void* o, float* lse, void* ws,
+                       size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then reads the status word a previous call left in
  * `ws`: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INDEX.  `code` (nullable)

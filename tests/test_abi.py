@@ -61,6 +61,17 @@ def test_window_fields_accepted(lib):
         assert lib.workspace_size(dims(lib, window=w, dilation=s), lib.MSA_SELECT) == 256
 
 
+def test_decode_workspace(lib):
+    """Decode keeps one index row per (sequence, group): a batch far beyond the
+    training path's index bound is still valid there."""
+    big = dims(lib, B=64, T=131072, Hq=32, Hkv=8, d=128, dp=64, topk=64)
+    assert lib.workspace_size(big, lib.MSA_FWD) == 0
+    ws = lib.workspace_size(big, lib.MSA_DECODE)
+    # status + pooled [B*Hp*nblk] fp32 + partials [B*Hkv*topk*G*(d+2)] fp32
+    assert ws >= 256 + 64 * 8 * 1024 * 4 + 64 * 8 * 64 * 4 * 130 * 4
+    assert ws % 256 == 0
+
+
 def test_workspace_sizes(lib):
     d = dims(lib)
     sel = lib.workspace_size(d, lib.MSA_SELECT)
