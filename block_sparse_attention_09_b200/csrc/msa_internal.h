@@ -44,13 +44,17 @@ WsLayout ws_layout(const Problem& p, int which);
 bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t e0, uint64_t e1, uint64_t e2,
                        uint64_t e3, uint32_t box0, uint32_t box2);
 
-// Query blocks per work-item range of the Main Branch kernels: the query-side
+// Query blocks per work-item range of the Main Branch kernels.  The query-side
 // rows one range touches (fp32 accumulators and gathered bf16 inputs of a
-// group) stay near 24 MB, well inside L2.
+// group) stay near 48 MB, inside L2; larger ranges mean fewer, longer work
+// items (less per-item setup).  At least four ranges per sequence keep the
+// items numerous enough to balance across the SMs on shorter sequences.
 inline int range_blocks(const Problem& p)
 {
     const long bytes_per_block = 128L * p.G * p.d * (4 + 2);
-    long rb = (24L << 20) / bytes_per_block;
+    long rb = (48L << 20) / bytes_per_block;
+    const long quarter = (p.nblk + 3) / 4;
+    if (rb > quarter) rb = quarter;
     if (rb < 1) rb = 1;
     if (rb > p.nblk) rb = p.nblk;
     return (int)rb;
