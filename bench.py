@@ -359,8 +359,8 @@ def main():
     B, T, Hq, Hkv, D = cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.d
     dims = msa.make_dims(B, T, Hq, Hkv, D, cfg.dp, cfg.topk)
     ws_sel = msa.workspace(dims, msa.MSA_SELECT, dev)
-    ws_fwd = msa.workspace(dims, msa.MSA_FWD, dev)
-    ws_bwd = msa.workspace(dims, msa.MSA_BWD, dev)
+    ws_fwd = msa.step_workspace(dims, dev)   # the backward reuses the forward's inverse index
+    ws_bwd = ws_fwd
     o = torch.empty_like(d["q"])
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
@@ -377,17 +377,18 @@ def main():
         if ev is not None:
             ev[2].record(stream)
         msa.bwd(inputs["q"], inputs["k"], inputs["v"], o, inputs["dout"], lse, idx, nsel, ws=ws_bwd,
-                out=(dq, dk, dv))
+                out=(dq, dk, dv), reuse_index=True)
         if ev is not None:
             ev[3].record(stream)
         return idx, nsel
 
-    # correctness guard on the timed configuration: every device status word clean
-    idx, nsel = step(d)
-    for ws in (ws_sel, ws_fwd, ws_bwd):
-        rc = msa.check_status(ws)
-        if rc != 0:
-            raise RuntimeError(f"device status {rc} on the benchmark workload")
+    # correctness guard on the timed configuration: every call's device status
+    # word clean (each call resets its status, so each is read right after it)
+    idx, nsel = msa.proxy_select(d["qp"], d["kp"], cfg.topk, ws=ws_sel, window=args.window,
+                                 dilation=args.dilation, check=True)
+    msa.fwd(d["q"], d["k"], d["v"], idx, nsel, ws=ws_fwd, out=(o, lse), check=True)
+    msa.bwd(d["q"], d["k"], d["v"], o, d["dout"], lse, idx, nsel, ws=ws_bwd, out=(dq, dk, dv), reuse_index=True,
+            check=True)
     f_proxy, f_fwd, f_bwd = flops_from_nsel(cfg, pair_count(cfg, nsel))
     f_step = f_proxy + f_fwd + f_bwd
 
@@ -486,7 +487,8 @@ def main():
                 ix, ns = msa.proxy_select(inp["qp"], inp["kp"], cfg.topk, ws=ws_sel, window=args.window,
                                           dilation=args.dilation)
                 msa.fwd(inp["q"], inp["k"], inp["v"], ix, ns, ws=ws_fwd, out=(oo, ll))
-                msa.bwd(inp["q"], inp["k"], inp["v"], oo, inp["dout"], ll, ix, ns, ws=ws_bwd, out=(qq, kk_, vv))
+                msa.bwd(inp["q"], inp["k"], inp["v"], oo, inp["dout"], ll, ix, ns, ws=ws_bwd, out=(qq, kk_, vv),
+                        reuse_index=True)
                 comp_done[sb].record(stream)
                 ds.wait_event(comp_done[sb])
                 with torch.cuda.stream(ds):               # this step's results

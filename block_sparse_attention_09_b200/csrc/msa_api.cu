@@ -128,6 +128,10 @@ int check_device()
 {
     int dev = 0, major = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MSA_ERR_DEVICE;
+    // bind the device's primary context to this host thread: tensor-map
+    // encoding needs a current context, and a caller's worker thread (an
+    // autograd engine thread, say) may not have one yet
+    if (cudaSetDevice(dev) != cudaSuccess) return MSA_ERR_DEVICE;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MSA_ERR_DEVICE;
     return major == 10 ? MSA_OK : MSA_ERR_DEVICE;
 }
@@ -181,8 +185,8 @@ int msa_proxy_select(const msa_dims* dims, const void* qp, const void* kp, int32
     return MSA_OK;
 }
 
-int msa_fwd(const msa_dims* dims, const void* q, const void* k, const void* v, const int32_t* idx,
-            const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes, void* stream)
+int msa_fwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v, const int32_t* idx,
+               const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes, void* stream, int flags)
 {
     Problem p;
     int rc = to_problem(dims, &p);
@@ -202,14 +206,21 @@ int msa_fwd(const msa_dims* dims, const void* q, const void* k, const void* v, c
     cudaStream_t st = (cudaStream_t)stream;
     uint32_t* status = (uint32_t*)((uint8_t*)ws + L.status);
     if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
-    if (launch_block_index(p, idx, nsel, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    if (!(flags & MSA_REUSE_INDEX) && launch_block_index(p, idx, nsel, ws, L, st) != cudaSuccess)
+        return MSA_ERR_LAUNCH;
     if (launch_fwd(p, q, k, v, tk, tv, idx, nsel, o, lse, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     return MSA_OK;
 }
 
-int msa_bwd(const msa_dims* dims, const void* q, const void* k, const void* v, const void* o, const void* dout,
-            const float* lse, const int32_t* idx, const int32_t* nsel, void* dq, void* dk, void* dv, void* ws,
-            size_t ws_bytes, void* stream)
+int msa_fwd(const msa_dims* dims, const void* q, const void* k, const void* v, const int32_t* idx,
+            const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes, void* stream)
+{
+    return msa_fwd_ex(dims, q, k, v, idx, nsel, o, lse, ws, ws_bytes, stream, 0);
+}
+
+int msa_bwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v, const void* o,
+               const void* dout, const float* lse, const int32_t* idx, const int32_t* nsel, void* dq, void* dk,
+               void* dv, void* ws, size_t ws_bytes, void* stream, int flags)
 {
     Problem p;
     int rc = to_problem(dims, &p);
@@ -230,9 +241,17 @@ int msa_bwd(const msa_dims* dims, const void* q, const void* k, const void* v, c
     cudaStream_t st = (cudaStream_t)stream;
     uint32_t* status = (uint32_t*)((uint8_t*)ws + L.status);
     if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
-    if (launch_block_index(p, idx, nsel, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    if (!(flags & MSA_REUSE_INDEX) && launch_block_index(p, idx, nsel, ws, L, st) != cudaSuccess)
+        return MSA_ERR_LAUNCH;
     if (launch_bwd(p, q, dout, tk, tv, o, lse, dq, dk, dv, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     return MSA_OK;
+}
+
+int msa_bwd(const msa_dims* dims, const void* q, const void* k, const void* v, const void* o, const void* dout,
+            const float* lse, const int32_t* idx, const int32_t* nsel, void* dq, void* dk, void* dv, void* ws,
+            size_t ws_bytes, void* stream)
+{
+    return msa_bwd_ex(dims, q, k, v, o, dout, lse, idx, nsel, dq, dk, dv, ws, ws_bytes, stream, 0);
 }
 
 int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q, const void* qp, const void* k,

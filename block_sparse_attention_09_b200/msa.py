@@ -25,6 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 MSA_SELECT, MSA_FWD, MSA_BWD, MSA_DECODE = 0, 1, 2, 3
+MSA_REUSE_INDEX = 1
 _ERR = {0: "ok", -1: "invalid dimensions", -2: "null pointer", -3: "misaligned pointer",
         -4: "workspace too small", -5: "CUDA launch failed", -6: "device wait timed out",
         -7: "device is not sm_100", -8: "tensor map encoding failed",
@@ -61,6 +62,10 @@ def _load():
     lib.msa_diag_umma.argtypes = [I, I, I, P, P, P, P, P]
     lib.msa_diag_wait_timeout.argtypes = [U64, P, P]
     lib.msa_set_kernel_events.argtypes = [I, P, P]
+    lib.msa_fwd_ex.argtypes = [D, P, P, P, P, P, P, P, P, SZ, P, I]
+    lib.msa_fwd_ex.restype = I
+    lib.msa_bwd_ex.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P, I]
+    lib.msa_bwd_ex.restype = I
     lib.msa_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.msa_decode.restype = I
     lib.msa_kernel_launches.argtypes = []
@@ -99,6 +104,12 @@ def workspace_size(dims: Dims, which: int) -> int:
 
 def workspace(dims: Dims, which: int, device) -> torch.Tensor:
     return torch.empty(max(workspace_size(dims, which), 256), dtype=torch.uint8, device=device)
+
+
+def step_workspace(dims: Dims, device) -> torch.Tensor:
+    """One workspace for a forward and the backward that reuses its index."""
+    n = max(workspace_size(dims, MSA_FWD), workspace_size(dims, MSA_BWD), 256)
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def check_status(ws: torch.Tensor, stream=None) -> int:
@@ -141,7 +152,7 @@ def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False, 
     return (idx, nsel, pool) if pooled else (idx, nsel)
 
 
-def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None):
+def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None, reuse_index=False):
     """Main Branch forward.  Returns (o bf16 [B,T,Hq,d], lse fp32 [B,Hq,T])."""
     _bf16(q, k, v)
     B, T, Hq, d = q.shape
@@ -154,15 +165,18 @@ def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=No
         o, lse = out
     if ws is None:
         ws = workspace(dims, MSA_FWD, q.device)
-    _check(LIB.msa_fwd(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(idx), _p(nsel), _p(o), _p(lse), _p(ws),
-                       ws.numel(), _stream(stream)), "msa_fwd")
+    _check(LIB.msa_fwd_ex(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(idx), _p(nsel), _p(o), _p(lse), _p(ws),
+                          ws.numel(), _stream(stream), MSA_REUSE_INDEX if reuse_index else 0), "msa_fwd")
     if check:
         _check(check_status(ws, stream), "msa_fwd (device)")
     return o, lse
 
 
-def bwd(q, k, v, o, dout, lse, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None):
-    """Main Branch backward.  Returns (dq, dk, dv), bf16."""
+def bwd(q, k, v, o, dout, lse, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None,
+        reuse_index=False):
+    """Main Branch backward.  Returns (dq, dk, dv), bf16.  reuse_index: ``ws``
+    already holds the inverse index of these idx/nsel from an earlier call on
+    the same workspace (e.g. the forward of the same step)."""
     _bf16(q, k, v, o, dout)
     B, T, Hq, d = q.shape
     topk = idx.shape[3]
@@ -173,8 +187,9 @@ def bwd(q, k, v, o, dout, lse, idx, nsel, scale=0.0, stream=None, ws=None, check
         dq, dk, dv = out
     if ws is None:
         ws = workspace(dims, MSA_BWD, q.device)
-    _check(LIB.msa_bwd(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(o), _p(dout), _p(lse), _p(idx),
-                       _p(nsel), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream)), "msa_bwd")
+    _check(LIB.msa_bwd_ex(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(o), _p(dout), _p(lse), _p(idx),
+                          _p(nsel), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream),
+                          MSA_REUSE_INDEX if reuse_index else 0), "msa_bwd")
     if check:
         _check(check_status(ws, stream), "msa_bwd (device)")
     return dq, dk, dv
@@ -188,15 +203,19 @@ class MSAAttention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, qp, kp, topk, scale=0.0):
         idx, nsel = proxy_select(qp, kp, topk)
-        o, lse = fwd(q, k, v, idx, nsel, scale)
+        B, T, Hq, d = q.shape
+        ws = step_workspace(make_dims(B, T, Hq, k.shape[2], d, 64, topk, scale), q.device)
+        o, lse = fwd(q, k, v, idx, nsel, scale, ws=ws)
         ctx.save_for_backward(q, k, v, o, lse, idx, nsel)
         ctx.scale = scale
+        ctx.ws = ws   # holds the inverse index for the backward
         return o
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, o, lse, idx, nsel = ctx.saved_tensors
-        dq, dk, dv = bwd(q, k, v, o, dout.contiguous(), lse, idx, nsel, ctx.scale)
+        dq, dk, dv = bwd(q, k, v, o, dout.contiguous(), lse, idx, nsel, ctx.scale, ws=ctx.ws, reuse_index=True)
+        ctx.ws = None
         return dq, dk, dv, None, None, None, None
 
 

@@ -186,6 +186,23 @@ MSA_API int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q,
                        const void* v, const void* kp, int32_t* idx, int32_t* nsel, void* o, float* lse, void* ws,
                        size_t ws_bytes, void* stream);
 
+/*
+ * msa_fwd / msa_bwd with flags.  MSA_REUSE_INDEX: the workspace already holds
+ * the block -> query inverse index of exactly these idx, nsel and dims, left
+ * there by an earlier msa_fwd_ex / msa_bwd_ex on the same workspace (both
+ * layouts keep the index at the same offsets, so one workspace of
+ * max(msa_workspace_size(MSA_FWD), msa_workspace_size(MSA_BWD)) bytes serves
+ * a forward and the backward that follows it); the call skips rebuilding it.
+ * Reusing an index built from different idx is undefined.  flags = 0 is
+ * msa_fwd / msa_bwd.
+ */
+enum msa_flags { MSA_REUSE_INDEX = 1 };
+MSA_API int msa_fwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v, const int32_t* idx,
+                       const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes, void* stream, int flags);
+MSA_API int msa_bwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, const int32_t* idx, const int32_t* nsel, void* dq,
+                       void* dk, void* dv, void* ws, size_t ws_bytes, void* stream, int flags);
+
 /* Synchronises `stream`, then reads the status word a previous call left in
  * `ws`: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INDEX.  `code` (nullable)
  * receives the raw device code (which wait or check failed). */
