@@ -1,0 +1,65 @@
+"""Host logic of bench.py, on CPU: the FLOP model against a brute-force count of
+the (query head, key) pairs the oracle's own selection reads, and the guard
+that reports recorded DRAM traffic only for unchanged kernel sources."""
+import hashlib
+import os
+import sys
+
+import numpy as np
+import torch
+
+import oracle as O
+from block_sparse_attention_09_b200.inputs import Config, make_inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_flop_model_counts_the_selected_pairs():
+    cfg = Config("flops", B=2, T=1000, Hq=4, Hkv=2, d=64, dp=32, topk=3)
+    inp = make_inputs(cfg, seed=51, exact_proxy=True, parts=["qp", "kp"])
+    m = O.Dims(B=cfg.B, T=cfg.T, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, dp=cfg.dp, topk=cfg.topk)
+    idx, nsel, _ = O.select(m, inp["qp"].float().numpy(), inp["kp"].float().numpy())
+    # brute force: keys j <= i of every selected block, per (b, group, i)
+    pairs = 0
+    for b in range(cfg.B):
+        for g in range(cfg.Hkv):
+            for i in range(cfg.T):
+                for n in idx[b, g, i, :nsel[b, g, i]]:
+                    pairs += min(128, i - 128 * int(n) + 1)
+    f_proxy, f_fwd, f_bwd = bench.flops_from_nsel(cfg, bench.pair_count(cfg, torch.from_numpy(nsel)))
+    assert f_fwd == 4.0 * cfg.d * cfg.G * pairs
+    assert f_bwd == 2.5 * f_fwd
+    # proxy: every key before the query's own block, for query tiles that rank
+    scored = 0
+    for qb in range((cfg.T + 127) // 128):
+        if qb + 1 > cfg.topk:
+            scored += min(128, cfg.T - 128 * qb) * 128 * qb
+    assert f_proxy == 2.0 * cfg.dp * scored * cfg.B * cfg.Hkv
+
+
+def test_recorded_traffic_needs_unchanged_sources(tmp_path, monkeypatch):
+    csrc = tmp_path / "block_sparse_attention_09_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "a.cu").write_bytes(b"kernel source")
+    (csrc / "b.h").write_bytes(b"header")
+    digest = hashlib.sha256(b"kernel source" + b"header").hexdigest()
+    (tmp_path / "profiles" / "dram_msa_w.md").write_text(
+        f"text\n```\ntraffic k1 123456 a.cu,b.h {digest}\ntraffic k2 5 a.cu 00\n```\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("k1", "w") == 123456.0
+    assert bench.recorded_traffic("k2", "w") is None          # hash differs
+    assert bench.recorded_traffic("k3", "w") is None          # no record
+    assert bench.recorded_traffic("k1", "other") is None      # no summary for the workload
+    (csrc / "a.cu").write_bytes(b"kernel source, edited")
+    assert bench.recorded_traffic("k1", "w") is None          # changed since the capture
+
+
+def test_workload_names():
+    cfg = Config("x", B=1, T=256, Hq=4, Hkv=1, d=64, dp=32, topk=2, bias="recency")
+    assert "recency" in bench.workload_name(cfg)
+    assert "window" not in bench.workload_name(cfg)
+    assert "forced window 4 blocks at dilation 2" in bench.workload_name(cfg, 4, 2)
+    assert np.isfinite(bench.measured_peaks()[0]["hbm_gbs"])
