@@ -118,6 +118,10 @@ __global__ void __launch_bounds__(1024) index_ptr_kernel(const int32_t* __restri
     if (t == 1023) out[nblk] = part[1023];
 }
 
+// The tile's queries that selected block n form one run of the block's token
+// list (ptr[n] + off[qb][n] onward), in ascending order: a warp writes it
+// from the tile's membership mask, lane l taking bit l of each 32-bit word, so
+// the stores of one word land on consecutive positions.
 __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t* __restrict__ idx,
                                                          const int32_t* __restrict__ nsel, int T, int topk,
                                                          int nblk, const int32_t* __restrict__ off,
@@ -127,25 +131,21 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t* __restri
     extern __shared__ uint32_t mask[];
     const int qb = blockIdx.x, bg = blockIdx.y;
     build_masks(mask, idx, nsel, T, topk, qb, bg);
-    const int t = threadIdx.x, i = qb * 128 + t;
-    if (i >= T) return;
-    const int64_t row = (int64_t)bg * T + i;
-    int ns = nsel[row];
-    ns = ns < 0 ? 0 : (ns > topk ? topk : ns);
-    const int32_t* sel = idx + row * topk;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t* offrow = off + ((int64_t)bg * nblk + qb) * nblk;
     const int32_t* p = ptr + (int64_t)bg * (nblk + 1);
     int32_t* out = tok + (int64_t)bg * T * topk;
-    const int w = t >> 5;
-    const uint32_t below = (1u << (t & 31)) - 1u;
-    int prev = -1;
-    for (int s = 0; s < ns; ++s) {
-        const int n = sel[s];
-        if (n < 0 || n > qb || n <= prev) continue;
-        prev = n;
-        int before = __popc(mask[n * 4 + w] & below);
-        for (int ww = 0; ww < w; ++ww) before += __popc(mask[n * 4 + ww]);
-        out[p[n] + offrow[n] + before] = i;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int n = warp; n <= qb; n += 4) {
+        const uint32_t m0 = mask[n * 4], m1 = mask[n * 4 + 1], m2 = mask[n * 4 + 2], m3 = mask[n * 4 + 3];
+        if ((m0 | m1 | m2 | m3) == 0u) continue;
+        int pos = p[n] + offrow[n];
+        const uint32_t mw[4] = {m0, m1, m2, m3};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            if ((mw[w] >> lane) & 1u) out[pos + __popc(mw[w] & below)] = qb * 128 + w * 32 + lane;
+            pos += __popc(mw[w]);
+        }
     }
 }
 

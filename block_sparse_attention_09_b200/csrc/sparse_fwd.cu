@@ -314,23 +314,19 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
 }
 
-// |q| per query row and max |k| per (b, group).  D/8 lanes per row.
+// |q| per query row; D/8 lanes per row (a streaming read of Q).
 template <int D>
-__global__ void __launch_bounds__(256) fwd_norms_kernel(const __nv_bfloat16* __restrict__ q,
-                                                        const __nv_bfloat16* __restrict__ k, int B, int T,
-                                                        int Hq, int Hkv, float* __restrict__ qn,
-                                                        uint32_t* __restrict__ kmax_bits)
+__global__ void __launch_bounds__(256) fwd_qnorm_kernel(const __nv_bfloat16* __restrict__ q, int B, int T, int Hq,
+                                                        float* __restrict__ qn)
 {
     constexpr int LPR = D / 8;
     const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t row = gt / LPR;
     const int sub = (int)(gt % LPR);
-    const int64_t nq = (int64_t)B * T * Hq, nk = (int64_t)B * T * Hkv;
-    const bool isq = row < nq, isk = !isq && row < nq + nk;
+    const bool ok = row < (int64_t)B * T * Hq;
     float ss = 0.f;
-    if (isq || isk) {
-        const __nv_bfloat16* src = isq ? q + row * D : k + (row - nq) * D;
-        const uint4 u = *reinterpret_cast<const uint4*>(src + sub * 8);
+    if (ok) {
+        const uint4 u = *reinterpret_cast<const uint4*>(q + row * D + sub * 8);
         const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -341,18 +337,55 @@ __global__ void __launch_bounds__(256) fwd_norms_kernel(const __nv_bfloat16* __r
     }
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if (sub == 0) {
-        if (isq) {
-            const int h = (int)(row % Hq);
-            const int64_t bi = row / Hq;
-            const int i = (int)(bi % T), b = (int)(bi / T);
-            qn[((int64_t)b * Hq + h) * T + i] = sqrtf(ss);
-        } else if (isk) {
-            const int64_t kr = row - nq;
-            const int gg = (int)(kr % Hkv);
-            const int b = (int)(kr / Hkv / T);
-            atomicMax(&kmax_bits[b * Hkv + gg], __float_as_uint(sqrtf(ss)));
+    if (ok && sub == 0) {
+        const int h = (int)(row % Hq);
+        const int64_t bi = row / Hq;
+        const int i = (int)(bi % T), b = (int)(bi / T);
+        qn[((int64_t)b * Hq + h) * T + i] = sqrtf(ss);
+    }
+}
+
+// max |k| per (b, group): grid (ceil(T / kKRows), B*Hkv); each CTA reduces its
+// rows to one value before a single atomic max (non-negative floats order like
+// their bits).
+constexpr int kKRows = 512;
+
+template <int D>
+__global__ void __launch_bounds__(256) fwd_kmax_kernel(const __nv_bfloat16* __restrict__ k, int T, int Hkv,
+                                                       uint32_t* __restrict__ kmax_bits)
+{
+    constexpr int LPR = D / 8, RPP = 256 / LPR;   // lanes per row, rows per pass
+    __shared__ float red[8];
+    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
+    const int sub = threadIdx.x % LPR, r = threadIdx.x / LPR;
+    float mx = 0.f;
+    // the same number of passes for every lane: the shuffles below need the
+    // whole warp, and rows past T are predicated off instead
+    for (int pass = 0; pass < kKRows / RPP; ++pass) {
+        const int t = blockIdx.x * kKRows + pass * RPP + r;
+        float ss = 0.f;
+        if (t < T) {
+            const uint4 u = *reinterpret_cast<const uint4*>(k + (((int64_t)b * T + t) * Hkv + g) * D + sub * 8);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                ss = fmaf(f.x, f.x, ss);
+                ss = fmaf(f.y, f.y, ss);
+            }
         }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        mx = fmaxf(mx, ss);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = red[0];
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+        atomicMax(&kmax_bits[bg], __float_as_uint(sqrtf(m)));
     }
 }
 
@@ -496,10 +529,11 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     if ((e = cudaMemsetAsync(lacc, 0, sizeof(float) * (size_t)pr.rows_q(), st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(nflag, 0, sizeof(int), st)) != cudaSuccess) return e;
 
-    const int64_t nrows = (int64_t)pr.B * pr.T * (pr.Hq + pr.Hkv);
-    const int64_t th = nrows * (D / 8);
-    fwd_norms_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(qb, kb, pr.B, pr.T, pr.Hq, pr.Hkv, qn,
-                                                                     (uint32_t*)kmax);
+    const int64_t th = (int64_t)pr.B * pr.T * pr.Hq * (D / 8);
+    fwd_qnorm_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(qb, pr.B, pr.T, pr.Hq, qn);
+    count_launches(1);
+    dim3 gk((unsigned)((pr.T + kKRows - 1) / kKRows), (unsigned)(pr.B * pr.Hkv));
+    fwd_kmax_kernel<D><<<gk, 256, 0, st>>>(kb, pr.T, pr.Hkv, (uint32_t*)kmax);
     count_launches(1);
 
     FwdParams p;
