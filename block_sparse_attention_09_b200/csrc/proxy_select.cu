@@ -9,10 +9,13 @@
 // stays in shared memory; proxy key tiles n = 0 .. qb-1 stream in through a
 // TMA ring two key blocks at a time; one thread issues tcgen05 MMAs (M=128
 // queries, N=256 keys, K=dp: at N=128 an accumulation chain of dependent
-// MMAs runs at half rate) into two TMEM accumulators; eight epilogue warps (one TMEM lane = one
+// MMAs runs at half rate) into two TMEM accumulators; eight pooling warps (one TMEM lane = one
 // query row each; two warps per lane quarter, one per key block of the
-// 256-key MMA) reduce each 128-column block to its max and feed the row's
-// selection.  The diagonal tile is needed only for the optional
+// 256-key MMA) reduce each 128-column block to its max, free the
+// accumulator and pass the maxima through a shared-memory ring to four
+// selection warps, which own the rows' selection state.  Pooling and
+// selection thus overlap, and the accumulator is handed back to the MMA as
+// soon as it has been read.  The diagonal tile is needed only for the optional
 // pooled-score output: the own block is always selected, so selection only
 // ranks blocks 0 .. qb-1, which every query of the tile sees in full.
 //
@@ -39,9 +42,10 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 320;             // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
+constexpr int kThreads = 448;             // warp 0: TMA, 1: MMA, 2-9: pooling, 10-13: selection
 constexpr uint32_t kTileBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle slab)
 constexpr int kPend = 10;                  // pending slots per row (merge once one row holds 8)
+constexpr int kRing = 4;                   // pairs of block maxima in flight from pooling to selection
 
 struct Params {
     int B, T, Hp, dp, nblk, topk;
@@ -195,25 +199,27 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     // pair k holds key blocks hi = ntiles-1-2k (nearest first) and lo = hi-1
     // (lo = -1 past the first block: that half is zero-filled and ignored)
 
-    // epilogue row of this thread (warps 2..5 own TMEM lane quarters 2,3,0,1)
-    const int r = ((warp & 3) << 5) | lane;
+    // row of this thread: a pooling warp reads TMEM lane quarter warp & 3;
+    // selection warp 10 + q owns rows 32q .. 32q + 31
+    const bool sel_warp = warp >= 10;
+    const int r = sel_warp ? ((warp - 10) << 5) | lane : ((warp & 3) << 5) | lane;
     const int i = qb * 128 + r;
-    const bool row_ok = (warp >= 2) && (warp < 6) && (i < p.T);   // the selection-owning warps
+    const bool row_ok = sel_warp && (i < p.T);
 
     const int hk = k1 > 0 ? k1 : 0;
     uint8_t* qp_tile = smem;
     uint8_t* kp_tiles = smem + kTileBytes;
     uint2* heap = (uint2*)(smem + kTileBytes * (1 + 2 * NSTAGE));   // [topk-1][128]
     uint2* pend = heap + (size_t)hk * 128;                             // [kPend][128]
-    float* xchg = (float*)(pend + kPend * 128);   // [2][128]: max of the farther block of a pair
-    uint64_t* bars = (uint64_t*)(xchg + 2 * 128);
+    float* pm = (float*)(pend + kPend * 128);    // [kRing][2][128]: block maxima (lo, hi) of a pair
+    uint64_t* bars = (uint64_t*)(pm + kRing * 2 * 128);
     uint64_t* full = bars;                     // [NSTAGE] TMA -> MMA
     uint64_t* empty = bars + NSTAGE;           // [NSTAGE] MMA -> TMA
     uint64_t* acc_full = bars + 2 * NSTAGE;    // [NACC] MMA -> epilogue
     uint64_t* acc_empty = acc_full + NACC;     // [NACC] epilogue -> MMA
-    uint64_t* xchg_full = acc_empty + NACC;    // [2] far-block warps -> selection warps
-    uint64_t* xchg_empty = xchg_full + 2;      // [2] selection warps -> far-block warps
-    uint64_t* qp_full = xchg_empty + 2;
+    uint64_t* pm_full = acc_empty + NACC;      // [kRing] pooling -> selection
+    uint64_t* pm_empty = pm_full + kRing;      // [kRing] selection -> pooling
+    uint64_t* qp_full = pm_empty + kRing;
     uint64_t* fin = qp_full + 1;               // MMA teardown drain
     uint32_t* tmem_hold = (uint32_t*)(fin + 1);
     volatile uint32_t* abort_flag = tmem_hold + 1;
@@ -231,7 +237,7 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int s = 0; s < NACC; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], 256); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&xchg_full[s], 128); mbar_init(&xchg_empty[s], 128); }
+        for (int s = 0; s < kRing; ++s) { mbar_init(&pm_full[s], 256); mbar_init(&pm_empty[s], 128); }
         mbar_init(qp_full, 1);
         mbar_init(fin, 1);
         *abort_flag = 0u;
@@ -290,9 +296,60 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
             umma_commit(fin);     // every MMA issued above has finished once this fires
             mbar_drain(fin, 0);
         }
-    } else {
-        // ---------------- epilogue: pool + select ----------------
+    } else if (!sel_warp) {
+        // ---------------- pooling: one 128-key block per warp and pair ----------------
+        // warps 2-5 reduce the nearer block of each pair (accumulator columns
+        // 128..255), warps 6-9 the farther one (columns 0..127), each on its
+        // TMEM lane quarter; the accumulator is released as soon as both
+        // maxima are in registers.
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
+        const bool near = warp < 6;
+        // max over one 128-key block, read from TMEM in two halves of 64
+        // columns (14 warps leave 128 registers a thread); the own block is
+        // cut at the query (causal)
+        auto block_max = [&](uint32_t ta, bool diag) -> float {
+            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t v[64];
+                tmem_ld32(ta + h * 64, v);
+                tmem_ld32(ta + h * 64 + 32, v + 32);
+                tmem_ld_wait();
+                if (diag) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (h * 64 + c > r) v[c] = __float_as_uint(-INFINITY);
+                }
+#pragma unroll
+                for (int c = 0; c < 64; c += 8) {
+                    m0 = fmax3(m0, __uint_as_float(v[c + 0]), __uint_as_float(v[c + 1]));
+                    m1 = fmax3(m1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                    m2 = fmax3(m2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
+                    m3 = fmax3(m3, __uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
+                }
+            }
+            return fmaxf(fmax3(m0, m1, m2), m3);
+        };
+        for (int k = 0; k < npairs; ++k) {
+            const int hi = ntiles - 1 - 2 * k, lo = hi - 1;
+            const int buf = k % NACC;
+            bool ok = mbar_wait(&acc_full[buf], (uint32_t)(k / NACC) & 1u, wc, code0 + 4);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 256u);
+            const float mx = near ? block_max(ta + 128, hi == qb) : (lo >= 0 ? block_max(ta, false) : -INFINITY);
+            tc_fence_before();
+            mbar_arrive(&acc_empty[buf]);   // the accumulator is free for pair k + NACC
+            const int slot = k % kRing;
+            if (k >= kRing) {
+                ok = mbar_wait(&pm_empty[slot], (uint32_t)(k / kRing - 1) & 1u, wc, code0 + 5);
+                if (!__all_sync(0xffffffffu, ok)) break;
+            }
+            pm[(slot * 2 + (near ? 1 : 0)) * 128 + r] = mx;
+            mbar_arrive(&pm_full[slot]);
+        }
+    } else {
+        // ---------------- selection: rows 32 (warp - 10) .. + 31 ----------------
         int cnt = 0, npend = 0;
         float tau = -INFINITY;   // score of the heap root once the heap is full
         auto merge_pending = [&]() {
@@ -305,30 +362,6 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
             }
             npend = 0;
             tau = __uint_as_float(heap[r].x);
-        };
-        // max over one 128-key block (TMEM columns col0 .. col0+127); the own
-        // block is cut at the query (causal)
-        auto block_max = [&](uint32_t ta, bool diag) -> float {
-            uint32_t v[128];
-            tmem_ld32(ta, v);
-            tmem_ld32(ta + 32, v + 32);
-            tmem_ld32(ta + 64, v + 64);
-            tmem_ld32(ta + 96, v + 96);
-            tmem_ld_wait();
-            if (diag) {
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c > r) v[c] = __float_as_uint(-INFINITY);
-            }
-            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; c += 8) {
-                m0 = fmax3(m0, __uint_as_float(v[c + 0]), __uint_as_float(v[c + 1]));
-                m1 = fmax3(m1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-                m2 = fmax3(m2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
-                m3 = fmax3(m3, __uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
-            }
-            return fmaxf(fmax3(m0, m1, m2), m3);
         };
         // blocks arrive in descending order: the next forced block below the own
         // one is a running pointer (-1 once all nf - 1 of them have passed)
@@ -351,53 +384,29 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
                 ++npend;
             }
         };
-        // warps 2-5 reduce the nearer block of each pair and own the selection
-        // state; warps 6-9 (same TMEM lane quarters) reduce the farther block
-        // and hand its max over through shared memory.
-        const bool sel_warp = warp < 6;
         for (int k = 0; k < npairs; ++k) {
             const int hi = ntiles - 1 - 2 * k, lo = hi - 1;
-            const int buf = k % NACC;
-            const uint32_t use = (uint32_t)(k / NACC);
-            bool ok = mbar_wait(&acc_full[buf], use & 1u, wc, code0 + 4);
+            const int slot = k % kRing;
+            const bool ok = mbar_wait(&pm_full[slot], (uint32_t)(k / kRing) & 1u, wc, code0 + 6);
             if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-            const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 256u);
-            // columns 0..127: block lo, 128..255: block hi
-            if (sel_warp) {
-                const float mhi = block_max(ta + 128, hi == qb);
-                tc_fence_before();
-                mbar_arrive(&acc_empty[buf]);   // the accumulator is free for pair k + NACC
-                ok = mbar_wait(&xchg_full[k & 1], (uint32_t)(k >> 1) & 1u, wc, code0 + 5);
-                if (!__all_sync(0xffffffffu, ok)) break;
-                const float mlo = xchg[(k & 1) * 128 + r];
-                mbar_arrive(&xchg_empty[k & 1]);
-                consume(hi, mhi);
-                if (lo >= 0) consume(lo, mlo);
-                // one vote per pair: at most two appends per pair, so a list
-                // holding 8 still has room for the next pair
-                if (need_heap && cnt == k1 && __any_sync(0xffffffffu, npend >= kPend - 2)) merge_pending();
-            } else {
-                const float mlo = lo >= 0 ? block_max(ta, false) : -INFINITY;
-                tc_fence_before();
-                mbar_arrive(&acc_empty[buf]);
-                if (k >= 2) {
-                    ok = mbar_wait(&xchg_empty[k & 1], (uint32_t)((k >> 1) - 1) & 1u, wc, code0 + 6);
-                    if (!__all_sync(0xffffffffu, ok)) break;
-                }
-                xchg[(k & 1) * 128 + r] = mlo;
-                mbar_arrive(&xchg_full[k & 1]);
-            }
+            const float mhi = pm[(slot * 2 + 1) * 128 + r], mlo = pm[slot * 2 * 128 + r];
+            mbar_arrive(&pm_empty[slot]);
+            consume(hi, mhi);
+            if (lo >= 0) consume(lo, mlo);
+            // one vote per pair: at most two appends per pair, so a list
+            // holding 8 still has room for the next pair
+            if (need_heap && cnt == k1 && __any_sync(0xffffffffu, npend >= kPend - 2)) merge_pending();
         }
-        if (sel_warp && need_heap && cnt == k1) merge_pending();
+        if (need_heap && cnt == k1) merge_pending();
         const bool go = __all_sync(0xffffffffu, !*abort_flag);
-        if (sel_warp && go) {
+        __syncwarp();   // each lane's heap column is read by the whole warp below
+        if (go) {
             if (need_heap) {
                 const int64_t row0 = (int64_t)bg * p.T + qb * 128;
                 if (p.topk <= 64)
-                    write_selection<2>(heap, k1, p.topk, p.dilation, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+                    write_selection<2>(heap, k1, p.topk, p.dilation, warp - 10, qb, p.T, row0, p.idx, p.nsel);
                 else
-                    write_selection<4>(heap, k1, p.topk, p.dilation, warp & 3, qb, p.T, row0, p.idx, p.nsel);
+                    write_selection<4>(heap, k1, p.topk, p.dilation, warp - 10, qb, p.T, row0, p.idx, p.nsel);
             } else if (row_ok) {
                 write_unranked(p.idx + ((int64_t)bg * p.T + i) * p.topk, p.nsel + (int64_t)bg * p.T + i, take_all,
                                qb, nf, p.dilation, p.topk);
@@ -433,8 +442,8 @@ cudaError_t launch_variant(const Problem& pr, const CUtensorMap& tm_qp, const CU
 size_t smem_bytes(int nstage, int topk)
 {
     const size_t k1 = (size_t)(topk > 1 ? topk - 1 : 0);
-    return 1024 + (size_t)kTileBytes * (1 + 2 * nstage) + k1 * 128 * 8 + (size_t)kPend * 128 * 8 + 2 * 128 * 4 +
-           32 * 8 + 16;
+    return 1024 + (size_t)kTileBytes * (1 + 2 * nstage) + k1 * 128 * 8 + (size_t)kPend * 128 * 8 +
+           (size_t)kRing * 2 * 128 * 4 + 32 * 8 + 16;
 }
 
 }  // namespace
