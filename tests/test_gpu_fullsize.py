@@ -1,5 +1,7 @@
 """Parity at the full workload sizes, in the launch configuration the
-benchmark times (whole tensors on the GPU, one call per phase).
+benchmark times (whole tensors on the GPU, one call per phase, one workspace
+shared by the forward and the backward, which reuses the forward's inverse
+index).
 
 The oracle cannot run every row at T = 128K, so it checks sampled outputs it
 computes one by one -- the selection of sampled queries (bit-exact: proxy
@@ -20,15 +22,17 @@ from parity_util import compare, f32, odims, to_dev
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
-@pytest.mark.parametrize("name,nsel_rows,nq_rows", [("32k", 256, 512), ("128k", 192, 384)])
+@pytest.mark.parametrize("name,nsel_rows,nq_rows", [("32k", 256, 512), ("128k", 192, 384), ("512k", 128, 256)])
 def test_full_size(name, nsel_rows, nq_rows):
     from block_sparse_attention_09_b200 import msa
     cfg = CONFIGS[name]
     inp = make_inputs(cfg, seed=11, exact_proxy=True)
     dev = to_dev(inp)
     idx, nsel = msa.proxy_select(dev["qp"], dev["kp"], cfg.topk, check=True)
-    o, lse = msa.fwd(dev["q"], dev["k"], dev["v"], idx, nsel, check=True)
-    dq, dk, dv = msa.bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, idx, nsel, check=True)
+    ws = msa.step_workspace(msa.make_dims(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.d, cfg.dp, cfg.topk), dev["q"].device)
+    o, lse = msa.fwd(dev["q"], dev["k"], dev["v"], idx, nsel, ws=ws, check=True)
+    dq, dk, dv = msa.bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, idx, nsel, ws=ws, check=True,
+                         reuse_index=True)
     torch.cuda.synchronize()
     g_idx, g_nsel = idx.cpu().numpy(), nsel.cpu().numpy()
     x = {k: v.float().numpy() for k, v in inp.items()}
