@@ -536,6 +536,11 @@ def main():
             "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
             "frac_of_burst": achieved / float(peaks.get("bf16_tflops", peak))}
 
+    phase_rates = {"proxy_select": f_proxy / (phase_ms["proxy_select"] * 1e-3) / 1e12,
+                   "fwd": f_fwd / (phase_ms["fwd"] * 1e-3) / 1e12,
+                   "bwd": f_bwd / (phase_ms["bwd"] * 1e-3) / 1e12,
+                   "fwd+bwd": (f_fwd + f_bwd) / ((phase_ms["fwd"] + phase_ms["bwd"]) * 1e-3) / 1e12}
+
     cpu = None
     if not args.no_cpu and world == 1:
         x = oracle_arrays(host)
@@ -557,11 +562,13 @@ def main():
         "frac_of_peak": tflops / float(peaks.get("bf16_tflops")),
         "flops_per_step": {"proxy": f_proxy, "fwd": f_fwd, "bwd": f_bwd},
         "phases_ms": phase_ms,
-        "phase_tflops": {"proxy_select": f_proxy / (phase_ms["proxy_select"] * 1e-3) / 1e12,
-                         "fwd": f_fwd / (phase_ms["fwd"] * 1e-3) / 1e12,
-                         "bwd": f_bwd / (phase_ms["bwd"] * 1e-3) / 1e12,
-                         "fwd+bwd": (f_fwd + f_bwd) / ((phase_ms["fwd"] + phase_ms["bwd"]) * 1e-3) / 1e12},
+        "phase_tflops": phase_rates,
         "kernel_ms": kern_ms,
+        # the same rates as fractions of the sustained bf16 peak (the proxy
+        # selection and the fwd+bwd pair are the two targets named for the path)
+        "phase_frac_of_peak": {k: v / peak for k, v in phase_rates.items()},
+        # tokens/s of the main branch alone (forward + backward, no selection)
+        "tokens_per_s_main": world * B * T / ((phase_ms["fwd"] + phase_ms["bwd"]) * 1e-3),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
