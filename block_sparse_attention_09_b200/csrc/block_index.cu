@@ -16,6 +16,8 @@
 //          ptr[n] + cnt[qb][n] + popcount(mask bits below t)
 // Selection entries outside [0, i/128], not strictly ascending, or rows
 // with nsel outside [1, topk] are skipped and flagged in the status word.
+// Only query tiles qb0 .. nblk-1 take part (rows before the first computed
+// query are not read): their cnt rows alone are written and scanned.
 #include "msa_device.cuh"
 #include "msa_internal.h"
 
@@ -50,11 +52,11 @@ __device__ bool build_masks(uint32_t* mask, const int32_t* idx, const int32_t* n
 
 __global__ void __launch_bounds__(128) index_count_kernel(const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ nsel, int T, int topk,
-                                                          int nblk, int32_t* __restrict__ cnt,
+                                                          int nblk, int qb0, int32_t* __restrict__ cnt,
                                                           uint32_t* status)
 {
     extern __shared__ uint32_t mask[];
-    const int qb = blockIdx.x, bg = blockIdx.y;
+    const int qb = qb0 + (int)blockIdx.x, bg = blockIdx.y;
     if (!build_masks(mask, idx, nsel, T, topk, qb, bg)) atomicOr(status + 1, 1u);
     int32_t* out = cnt + ((int64_t)bg * nblk + qb) * nblk;
     for (int n = threadIdx.x; n <= qb; n += blockDim.x)
@@ -62,10 +64,11 @@ __global__ void __launch_bounds__(128) index_count_kernel(const int32_t* __restr
                  __popc(mask[n * 4 + 3]);
 }
 
-// cnt[bg][qb][n] for qb >= n  ->  exclusive prefix over qb; tot[bg][n] = sum.
-// Block (32 x 32): x = block id within a group of 32, y = segment of qb.
+// cnt[bg][qb][n] for qb >= max(n, qb0)  ->  exclusive prefix over qb;
+// tot[bg][n] = sum.  Block (32 x 32): x = block id within a group of 32,
+// y = segment of qb.
 __global__ void __launch_bounds__(1024) index_scan_kernel(int32_t* __restrict__ cnt,
-                                                          int32_t* __restrict__ tot, int nblk)
+                                                          int32_t* __restrict__ tot, int nblk, int qb0)
 {
     __shared__ int seg[32][33];
     const int n0 = blockIdx.x * 32;
@@ -77,14 +80,14 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int32_t* __restrict__ 
     int32_t* col = cnt + (int64_t)bg * nblk * nblk + n;
     int s = 0;
     if (n < nblk)
-        for (int q = max(q0, n); q < q1; ++q) s += col[(int64_t)q * nblk];
+        for (int q = max(q0, max(n, qb0)); q < q1; ++q) s += col[(int64_t)q * nblk];
     seg[threadIdx.y][threadIdx.x] = s;
     __syncthreads();
     int base = 0;
     for (int y = 0; y < (int)threadIdx.y; ++y) base += seg[y][threadIdx.x];
     if (n < nblk) {
         int run = base;
-        for (int q = max(q0, n); q < q1; ++q) {
+        for (int q = max(q0, max(n, qb0)); q < q1; ++q) {
             const int c = col[(int64_t)q * nblk];
             col[(int64_t)q * nblk] = run;
             run += c;
@@ -124,12 +127,12 @@ __global__ void __launch_bounds__(1024) index_ptr_kernel(const int32_t* __restri
 // the stores of one word land on consecutive positions.
 __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t* __restrict__ idx,
                                                          const int32_t* __restrict__ nsel, int T, int topk,
-                                                         int nblk, const int32_t* __restrict__ off,
+                                                         int nblk, int qb0, const int32_t* __restrict__ off,
                                                          const int32_t* __restrict__ ptr,
                                                          int32_t* __restrict__ tok)
 {
     extern __shared__ uint32_t mask[];
-    const int qb = blockIdx.x, bg = blockIdx.y;
+    const int qb = qb0 + (int)blockIdx.x, bg = blockIdx.y;
     build_masks(mask, idx, nsel, T, topk, qb, bg);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int32_t* offrow = off + ((int64_t)bg * nblk + qb) * nblk;
@@ -171,15 +174,15 @@ cudaError_t launch_block_index(const Problem& pr, const int32_t* idx, const int3
                                  (int)mask_bytes);
         if (e != cudaSuccess) return e;
     }
-    dim3 g1(pr.nblk, BH);
-    index_count_kernel<<<g1, 128, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, cnt, status);
+    dim3 g1(pr.nblk - pr.qb0, BH);   // the computed query tiles
+    index_count_kernel<<<g1, 128, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, pr.qb0, cnt, status);
     count_launches(1);
     dim3 g2((pr.nblk + 31) / 32, BH), b2(32, 32);
-    index_scan_kernel<<<g2, b2, 0, st>>>(cnt, tot, pr.nblk);
+    index_scan_kernel<<<g2, b2, 0, st>>>(cnt, tot, pr.nblk, pr.qb0);
     count_launches(1);
     index_ptr_kernel<<<BH, 1024, 0, st>>>(tot, ptr, pr.nblk);
     count_launches(1);
-    index_fill_kernel<<<g1, 128, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, cnt, ptr, tok);
+    index_fill_kernel<<<g1, 128, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, pr.qb0, cnt, ptr, tok);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -113,12 +113,17 @@ int to_problem(const msa_dims* d, Problem* p, bool decode = false)
     if (d->dp < 8 || d->dp > 64 || d->dp % 8 != 0) return MSA_ERR_INVALID_DIMS;
     if (!isfinite(d->scale)) return MSA_ERR_INVALID_DIMS;
     if (d->window < 0 || d->window > d->topk || d->dilation < 0 || d->dilation > kMaxT) return MSA_ERR_INVALID_DIMS;
+    // first computed query row: a block boundary inside [0, T]; decode has one query per sequence
+    if (d->q_begin < 0 || d->q_begin % kBlock != 0 || d->q_begin > d->T || (decode && d->q_begin != 0))
+        return MSA_ERR_INVALID_DIMS;
     p->B = d->B; p->T = d->T; p->Hq = d->Hq; p->Hkv = d->Hkv; p->Hp = d->Hp;
     p->d = d->d; p->dp = d->dp; p->topk = d->topk;
     p->nblk = (d->T + kBlock - 1) / kBlock;
     p->window = d->window > 0 ? d->window : 1;
     p->dilation = d->dilation > 0 ? d->dilation : 1;
     p->G = G;
+    p->q0 = d->q_begin;
+    p->qb0 = d->q_begin / kBlock;
     p->scale = d->scale != 0.f ? d->scale : 1.0f / sqrtf((float)d->d);
     if (!decode && (int64_t)p->B * p->Hp * p->T * p->topk > (int64_t)INT32_MAX) return MSA_ERR_INVALID_DIMS;
     return MSA_OK;
@@ -145,7 +150,7 @@ int check_ws(const Problem& p, int which, void* ws, size_t ws_bytes, WsLayout* L
     return MSA_OK;
 }
 
-bool empty(const Problem& p) { return p.B == 0 || p.T == 0; }
+bool empty(const Problem& p) { return p.B == 0 || p.T == 0 || p.q0 >= p.T; }
 
 }  // namespace
 
@@ -227,6 +232,16 @@ int msa_bwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v
     if (rc != MSA_OK) return rc;
     WsLayout L;
     if ((rc = check_ws(p, MSA_BWD, ws, ws_bytes, &L)) != MSA_OK) return rc;
+    if (p.B > 0 && p.T > 0 && p.q0 >= p.T) {
+        // no query row computed: the partial dK, dV are zero
+        if (!dk || !dv) return MSA_ERR_NULL_PTR;
+        if ((rc = check_device()) != MSA_OK) return rc;
+        const size_t bytes = (size_t)p.B * p.T * p.Hkv * p.d * ((flags & MSA_DKV_F32) ? 4 : 2);
+        if (cudaMemsetAsync(dk, 0, bytes, (cudaStream_t)stream) != cudaSuccess ||
+            cudaMemsetAsync(dv, 0, bytes, (cudaStream_t)stream) != cudaSuccess)
+            return MSA_ERR_LAUNCH;
+        return MSA_OK;
+    }
     if (empty(p)) return MSA_OK;
     if (!q || !k || !v || !o || !dout || !lse || !idx || !nsel || !dq || !dk || !dv) return MSA_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
@@ -243,7 +258,8 @@ int msa_bwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v
     if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     if (!(flags & MSA_REUSE_INDEX) && launch_block_index(p, idx, nsel, ws, L, st) != cudaSuccess)
         return MSA_ERR_LAUNCH;
-    if (launch_bwd(p, q, dout, tk, tv, o, lse, dq, dk, dv, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    if (launch_bwd(p, q, dout, tk, tv, o, lse, dq, dk, dv, (flags & MSA_DKV_F32) != 0, ws, L, st) != cudaSuccess)
+        return MSA_ERR_LAUNCH;
     return MSA_OK;
 }
 
@@ -274,6 +290,17 @@ int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q, const v
     if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     if (launch_decode(p, lens, q, qp, k, v, kp, idx, nsel, o, lse, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     return MSA_OK;
+}
+
+int msa_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream)
+{
+    if (n < 0 || n % 8 != 0) return MSA_ERR_INVALID_DIMS;
+    if (n == 0) return MSA_OK;
+    if (!src || !dst) return MSA_ERR_NULL_PTR;
+    if (!aligned(src, 16) || !aligned(dst, 16)) return MSA_ERR_MISALIGNED;
+    int rc = check_device();
+    if (rc != MSA_OK) return rc;
+    return launch_f32_to_bf16(src, dst, n, (cudaStream_t)stream) == cudaSuccess ? MSA_OK : MSA_ERR_LAUNCH;
 }
 
 int msa_check_status(const void* ws, void* stream, uint32_t* code)

@@ -296,25 +296,28 @@ struct RangeItem {
     int bg, n, beg, count;   // beg: offset into the group's token list
 };
 
-__host__ __device__ inline int range_items_per_group(int nblk, int RB)
+__host__ __device__ inline int range_items_per_group(int nblk, int RB, int qb0)
 {
     int total = 0;
-    for (int R = 0; R * RB < nblk; ++R) total += min(nblk, (R + 1) * RB);
+    for (int R = 0; qb0 + R * RB < nblk; ++R) total += min(nblk, qb0 + (R + 1) * RB);
     return total;
 }
 
-MSA_DEV RangeItem range_item(int x, int nblk, int RB, int per_group, const int32_t* ptr, const int32_t* off)
+// Ranges cover the query blocks qb0 .. nblk-1 (the queries computed); range R
+// holds the items of KV blocks 0 .. qe-1.
+MSA_DEV RangeItem range_item(int x, int nblk, int RB, int qb0, int per_group, const int32_t* ptr,
+                             const int32_t* off)
 {
     RangeItem it;
     it.bg = x / per_group;
     int rem = x % per_group, R = 0;
     for (;;) {
-        const int nv = min(nblk, (R + 1) * RB);
+        const int nv = min(nblk, qb0 + (R + 1) * RB);
         if (rem < nv) break;
         rem -= nv;
         ++R;
     }
-    const int n = rem, qs = R * RB, qe = min(nblk, (R + 1) * RB);
+    const int n = rem, qs = qb0 + R * RB, qe = min(nblk, qb0 + (R + 1) * RB);
     const int32_t* pp = ptr + (int64_t)it.bg * (nblk + 1);
     const int32_t* o = off + (int64_t)it.bg * nblk * nblk;
     const int base = pp[n];
@@ -324,6 +327,17 @@ MSA_DEV RangeItem range_item(int x, int nblk, int RB, int per_group, const int32
     it.beg = base + start;
     it.count = end - start;
     return it;
+}
+
+// Active query row r (0 .. B*(T-q0)*Hq - 1: the rows q0 .. T-1 of every batch
+// and head) -> its flat index (b*T + i)*Hq + h in a [B][T][Hq] tensor.
+MSA_DEV int64_t active_row(int64_t r, int T, int Hq, int q0)
+{
+    const int h = (int)(r % Hq);
+    const int64_t bi = r / Hq;
+    const int Tq = T - q0;
+    const int i = q0 + (int)(bi % Tq), b = (int)(bi / Tq);
+    return ((int64_t)b * T + i) * Hq + h;
 }
 
 // ---------------------------------------------------------------- math

@@ -24,8 +24,11 @@ enum KernelId : uint32_t { kKidProxy = 1, kKidFwd = 2, kKidBwd = 3, kKidDiag = 4
 struct Problem {
     int B, T, Hq, Hkv, Hp, d, dp, topk, nblk, G;
     int window, dilation;   // forced block pattern of the selection (>= 1)
+    int q0, qb0;            // first query row computed, and its block (q0 = 128 qb0)
     float scale;
     int64_t rows_q() const { return (int64_t)B * T * Hq; }
+    // query rows computed: rows q0 .. T-1 of every batch and head
+    int64_t rows_q_active() const { return (int64_t)B * (T - q0) * Hq; }
 };
 
 // Byte offsets of the workspace regions.
@@ -53,7 +56,7 @@ inline int range_blocks(const Problem& p)
 {
     const long bytes_per_block = 128L * p.G * p.d * (4 + 2);
     long rb = (48L << 20) / bytes_per_block;
-    const long quarter = (p.nblk + 3) / 4;
+    const long quarter = (p.nblk - p.qb0 + 3) / 4;
     if (rb > quarter) rb = quarter;
     if (rb < 1) rb = 1;
     if (rb > p.nblk) rb = p.nblk;
@@ -101,9 +104,13 @@ cudaError_t launch_fwd(const Problem& p, const void* q, const void* k, const voi
                        const int32_t* nsel, void* o, float* lse, void* ws, const WsLayout& L,
                        cudaStream_t st);
 
+// dkv_f32: dk, dv are fp32 and receive the unrounded sums
 cudaError_t launch_bwd(const Problem& p, const void* q, const void* dout, const CUtensorMap& tm_k,
                        const CUtensorMap& tm_v, const void* o, const float* lse, void* dq, void* dk,
-                       void* dv, void* ws, const WsLayout& L, cudaStream_t st);
+                       void* dv, bool dkv_f32, void* ws, const WsLayout& L, cudaStream_t st);
+
+// dst = bf16(src), n elements (a multiple of 8)
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t st);
 
 cudaError_t launch_diag_umma(int mode, int N, int K, const void* A, const void* B, float* D,
                              uint32_t* status, cudaStream_t st);

@@ -49,6 +49,7 @@ constexpr int kRing = 4;                   // pairs of block maxima in flight fr
 
 struct Params {
     int B, T, Hp, dp, nblk, topk;
+    int qb0;                // first query tile computed (earlier tiles are skipped)
     int window, dilation;   // forced blocks: qb, qb - dilation, ... (window of them)
     int32_t* idx;
     int32_t* nsel;
@@ -185,9 +186,11 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // group by group, heaviest (largest qb) tiles first within a group
-    const int bg = (int)(blockIdx.x / p.nblk);
-    const int qb = p.nblk - 1 - (int)(blockIdx.x % p.nblk);
+    // group by group, heaviest (largest qb) tiles first within a group; only
+    // the tiles qb0 .. nblk-1 are launched
+    const int nq = p.nblk - p.qb0;
+    const int bg = (int)(blockIdx.x / nq);
+    const int qb = p.nblk - 1 - (int)(blockIdx.x % nq);
     const int b = bg / p.Hp, g = bg % p.Hp;
     const int nf = WINDOW ? min(p.window, qb / p.dilation + 1) : 1;   // forced blocks that exist
     const int k1 = p.topk - nf;                            // slots ranked by pooled score
@@ -431,7 +434,7 @@ cudaError_t launch_variant(const Problem& pr, const CUtensorMap& tm_qp, const CU
     auto kern = proxy_select_kernel<NSTAGE, WINDOW>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)(pr.nblk * pr.B * pr.Hp);
+    const unsigned grid = (unsigned)((pr.nblk - pr.qb0) * pr.B * pr.Hp);
     trace_begin(kTraceProxy, st);
     kern<<<grid, kThreads, smem, st>>>(tm_qp, tm_kp, p);
     count_launches(1);
@@ -452,7 +455,7 @@ cudaError_t launch_proxy_select(const Problem& pr, const CUtensorMap& tm_qp, con
                                 int32_t* idx, int32_t* nsel, float* pooled, uint32_t* status,
                                 cudaStream_t st)
 {
-    Params p{pr.B, pr.T, pr.Hp, pr.dp, pr.nblk, pr.topk, pr.window, pr.dilation, idx, nsel, pooled, status};
+    Params p{pr.B, pr.T, pr.Hp, pr.dp, pr.nblk, pr.topk, pr.qb0, pr.window, pr.dilation, idx, nsel, pooled, status};
     // All of TMEM per CTA: at least 120 KB of shared memory keeps one CTA per SM.
     const bool win = pr.window > 1;
     const size_t s4 = smem_bytes(4, pr.topk);

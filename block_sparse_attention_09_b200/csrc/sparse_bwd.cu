@@ -39,7 +39,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct BwdParams {
     int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
-    int RB, per_group;   // query blocks per range; work items per (b, group)
+    int RB, qb0, per_group;   // query blocks per range; first query block; work items per (b, group)
     float c1;      // scale * log2(e)
     float scale;
     const __nv_bfloat16* q;
@@ -85,7 +85,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const RangeItem item = range_item((int)blockIdx.x, p.nblk, p.RB, p.per_group, p.ptr, p.off);
+    const RangeItem item = range_item((int)blockIdx.x, p.nblk, p.RB, p.qb0, p.per_group, p.ptr, p.off);
     const int n = item.n, bg = item.bg;
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int G = 1 << p.lgG;
@@ -476,17 +476,19 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
 }
 
-// D_i = dO_i . O_i per query row (bf16 inputs, fp32 sum); D/8 lanes per row.
+// D_i = dO_i . O_i per computed query row (rows q0 .. T-1; bf16 inputs, fp32
+// sum); D/8 lanes per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dsum_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout, int B, int T,
-                                                       int Hq, float* __restrict__ dsum)
+                                                       int Hq, int q0, float* __restrict__ dsum)
 {
     constexpr int LPR = D / 8;
     const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t row = gt / LPR;
+    const int64_t ar = gt / LPR;
     const int sub = (int)(gt % LPR);
-    const bool ok = row < (int64_t)B * T * Hq;
+    const bool ok = ar < (int64_t)B * (T - q0) * Hq;
+    const int64_t row = ok ? active_row(ar, T, Hq, q0) : 0;
     float s = 0.f;
     if (ok) {
         const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + sub * 8);
@@ -526,25 +528,47 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __rest
     *reinterpret_cast<uint4*>(dq + x * 8) = u;
 }
 
+// The computed rows (q0 .. T-1) of the fp32 dQ accumulator -> bf16 dQ.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_rows_kernel(const float* __restrict__ acc,
+                                                          __nv_bfloat16* __restrict__ dq, int B, int T, int Hq,
+                                                          int q0)
+{
+    constexpr int LPR = D / 8;
+    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t ar = gt / LPR;
+    if (ar >= (int64_t)B * (T - q0) * Hq) return;
+    const int64_t x = active_row(ar, T, Hq, q0) * D + (gt % LPR) * 8;
+    const float4 a = *reinterpret_cast<const float4*>(acc + x);
+    const float4 c = *reinterpret_cast<const float4*>(acc + x + 4);
+    uint4 u;
+    u.x = pack_bf16x2(a.x, a.y);
+    u.y = pack_bf16x2(a.z, a.w);
+    u.z = pack_bf16x2(c.x, c.y);
+    u.w = pack_bf16x2(c.z, c.w);
+    *reinterpret_cast<uint4*>(dq + x) = u;
+}
+
 template <int D>
 cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, const CUtensorMap& tm_k,
                          const CUtensorMap& tm_v, const void* o, const float* lse, void* dq, void* dk,
-                         void* dv, void* ws, const WsLayout& L, cudaStream_t st)
+                         void* dv, bool dkv_f32, void* ws, const WsLayout& L, cudaStream_t st)
 {
     uint8_t* w = (uint8_t*)ws;
     float* dsum = (float*)(w + L.dsum);
     float* dqacc = (float*)(w + L.dqacc);
-    float* dkacc = (float*)(w + L.dkacc);
-    float* dvacc = (float*)(w + L.dvacc);
+    // fp32 dK/dV outputs are accumulated in place
+    float* dkacc = dkv_f32 ? (float*)dk : (float*)(w + L.dkacc);
+    float* dvacc = dkv_f32 ? (float*)dv : (float*)(w + L.dvacc);
     const size_t kv_elems = (size_t)pr.B * pr.T * pr.Hkv * D;
     cudaError_t e;
     if ((e = cudaMemsetAsync(dqacc, 0, sizeof(float) * (size_t)pr.rows_q() * D, st)) != cudaSuccess)
         return e;
     if ((e = cudaMemsetAsync(dkacc, 0, sizeof(float) * kv_elems, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dvacc, 0, sizeof(float) * kv_elems, st)) != cudaSuccess) return e;
-    const int64_t th = pr.rows_q() * (D / 8);
+    const int64_t th = pr.rows_q_active() * (D / 8);
     bwd_dsum_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(
-        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, dsum);
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, pr.q0, dsum);
     count_launches(1);
 
     BwdParams p;
@@ -565,7 +589,8 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     p.dvacc = dvacc;
     p.status = (uint32_t*)(w + L.status);
     p.RB = range_blocks(pr);
-    p.per_group = range_items_per_group(pr.nblk, p.RB);
+    p.qb0 = pr.qb0;
+    p.per_group = range_items_per_group(pr.nblk, p.RB, pr.qb0);
     const size_t smem = BwdSmem<D>::kTotal;
     if ((e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
@@ -574,14 +599,17 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     bwd_main_kernel<D><<<(unsigned)(p.per_group * pr.B * pr.Hkv), kWarps * 32, smem, st>>>(tm_k, tm_v, p);
     count_launches(1);
     trace_end(kTraceBwdMain, st);
-    const int64_t n8 = pr.rows_q() * D / 8;
-    bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dqacc, (__nv_bfloat16*)dq, n8);
+    const int64_t n8 = pr.rows_q_active() * D / 8;
+    bwd_dq_rows_kernel<D><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dqacc, (__nv_bfloat16*)dq, pr.B, pr.T,
+                                                                          pr.Hq, pr.q0);
     count_launches(1);
-    const int64_t k8 = (int64_t)kv_elems / 8;
-    bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dkacc, (__nv_bfloat16*)dk, k8);
-    count_launches(1);
-    bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dvacc, (__nv_bfloat16*)dv, k8);
-    count_launches(1);
+    if (!dkv_f32) {
+        const int64_t k8 = (int64_t)kv_elems / 8;
+        bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dkacc, (__nv_bfloat16*)dk, k8);
+        count_launches(1);
+        bwd_dq_convert_kernel<<<(unsigned)((k8 + 255) / 256), 256, 0, st>>>(dvacc, (__nv_bfloat16*)dv, k8);
+        count_launches(1);
+    }
     return cudaGetLastError();
 }
 
@@ -589,10 +617,18 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
 
 cudaError_t launch_bwd(const Problem& pr, const void* q, const void* dout, const CUtensorMap& tm_k,
                        const CUtensorMap& tm_v, const void* o, const float* lse, void* dq, void* dk,
-                       void* dv, void* ws, const WsLayout& L, cudaStream_t st)
+                       void* dv, bool dkv_f32, void* ws, const WsLayout& L, cudaStream_t st)
 {
-    if (pr.d == 64) return launch_bwd_d<64>(pr, q, dout, tm_k, tm_v, o, lse, dq, dk, dv, ws, L, st);
-    return launch_bwd_d<128>(pr, q, dout, tm_k, tm_v, o, lse, dq, dk, dv, ws, L, st);
+    if (pr.d == 64) return launch_bwd_d<64>(pr, q, dout, tm_k, tm_v, o, lse, dq, dk, dv, dkv_f32, ws, L, st);
+    return launch_bwd_d<128>(pr, q, dout, tm_k, tm_v, o, lse, dq, dk, dv, dkv_f32, ws, L, st);
+}
+
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t st)
+{
+    const int64_t n8 = n / 8;
+    bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(src, (__nv_bfloat16*)dst, n8);
+    count_launches(1);
+    return cudaGetLastError();
 }
 
 }  // namespace msa

@@ -37,7 +37,7 @@ constexpr float kUnderflow = 5.421010862427522e-20f;   // 2^-64: row sums below 
 
 struct FwdParams {
     int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
-    int RB, per_group;   // query blocks per range; work items per (b, group)
+    int RB, qb0, per_group;   // query blocks per range; first query block; work items per (b, group)
     float c1;        // scale * log2(e)
     float bound;     // |scale| * log2(e)
     const __nv_bfloat16* q;
@@ -61,7 +61,7 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const RangeItem item = range_item((int)blockIdx.x, p.nblk, p.RB, p.per_group, p.ptr, p.off);
+    const RangeItem item = range_item((int)blockIdx.x, p.nblk, p.RB, p.qb0, p.per_group, p.ptr, p.off);
     const int n = item.n, bg = item.bg;
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int G = 1 << p.lgG;
@@ -314,16 +314,18 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
 }
 
-// |q| per query row; D/8 lanes per row (a streaming read of Q).
+// |q| per computed query row (rows q0 .. T-1); D/8 lanes per row (a
+// streaming read of Q).
 template <int D>
 __global__ void __launch_bounds__(256) fwd_qnorm_kernel(const __nv_bfloat16* __restrict__ q, int B, int T, int Hq,
-                                                        float* __restrict__ qn)
+                                                        int q0, float* __restrict__ qn)
 {
     constexpr int LPR = D / 8;
     const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t row = gt / LPR;
+    const int64_t ar = gt / LPR;
     const int sub = (int)(gt % LPR);
-    const bool ok = row < (int64_t)B * T * Hq;
+    const bool ok = ar < (int64_t)B * (T - q0) * Hq;
+    const int64_t row = ok ? active_row(ar, T, Hq, q0) : 0;
     float ss = 0.f;
     if (ok) {
         const uint4 u = *reinterpret_cast<const uint4*>(q + row * D + sub * 8);
@@ -389,22 +391,24 @@ __global__ void __launch_bounds__(256) fwd_kmax_kernel(const __nv_bfloat16* __re
     }
 }
 
-// O = O_acc / l (bf16), L = bound + log(l); rows whose l underflowed are listed.
+// O = O_acc / l (bf16), L = bound + log(l) for the computed rows (q0 ..
+// T-1); rows whose l underflowed are listed.
 template <int D>
 __global__ void __launch_bounds__(256) fwd_finalize_kernel(const float* __restrict__ oacc,
                                                            const float* __restrict__ lacc,
                                                            const float* __restrict__ qn,
                                                            const float* __restrict__ kmax, int B, int T,
-                                                           int Hq, int Hkv, float abs_scale,
+                                                           int Hq, int Hkv, int q0, float abs_scale,
                                                            __nv_bfloat16* __restrict__ o,
                                                            float* __restrict__ lse, int* nflag,
                                                            int* flags)
 {
     constexpr int LPR = D / 8;
     const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t row = gt / LPR;   // (b*T + i)*Hq + h
+    const int64_t ar = gt / LPR;
     const int sub = (int)(gt % LPR);
-    if (row >= (int64_t)B * T * Hq) return;
+    if (ar >= (int64_t)B * (T - q0) * Hq) return;
+    const int64_t row = active_row(ar, T, Hq, q0);   // (b*T + i)*Hq + h
     const int h = (int)(row % Hq);
     const int64_t bi = row / Hq;
     const int i = (int)(bi % T), b = (int)(bi / T);
@@ -529,8 +533,8 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     if ((e = cudaMemsetAsync(lacc, 0, sizeof(float) * (size_t)pr.rows_q(), st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(nflag, 0, sizeof(int), st)) != cudaSuccess) return e;
 
-    const int64_t th = (int64_t)pr.B * pr.T * pr.Hq * (D / 8);
-    fwd_qnorm_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(qb, pr.B, pr.T, pr.Hq, qn);
+    const int64_t th = pr.rows_q_active() * (D / 8);
+    fwd_qnorm_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(qb, pr.B, pr.T, pr.Hq, pr.q0, qn);
     count_launches(1);
     dim3 gk((unsigned)((pr.T + kKRows - 1) / kKRows), (unsigned)(pr.B * pr.Hkv));
     fwd_kmax_kernel<D><<<gk, 256, 0, st>>>(kb, pr.T, pr.Hkv, (uint32_t*)kmax);
@@ -549,7 +553,8 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     p.qn = qn; p.kmax = kmax; p.oacc = oacc; p.lacc = lacc;
     p.status = (uint32_t*)(w + L.status);
     p.RB = range_blocks(pr);
-    p.per_group = range_items_per_group(pr.nblk, p.RB);
+    p.qb0 = pr.qb0;
+    p.per_group = range_items_per_group(pr.nblk, p.RB, pr.qb0);
     const size_t smem = (size_t)(2 + kQStages) * 128 * D * 2 + 128 * D * 4 + 2048 + 32 * 8;
     if ((e = cudaFuncSetAttribute(fwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
@@ -559,9 +564,9 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     count_launches(1);
     trace_end(kTraceFwdMain, st);
 
-    const int64_t fth = (int64_t)pr.rows_q() * (D / 8);
+    const int64_t fth = pr.rows_q_active() * (D / 8);
     fwd_finalize_kernel<D><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(
-        oacc, lacc, qn, kmax, pr.B, pr.T, pr.Hq, pr.Hkv, fabsf(pr.scale), (__nv_bfloat16*)o, lse, nflag,
+        oacc, lacc, qn, kmax, pr.B, pr.T, pr.Hq, pr.Hkv, pr.q0, fabsf(pr.scale), (__nv_bfloat16*)o, lse, nflag,
         flags);
     count_launches(1);
     fwd_fallback_kernel<D><<<148, 128, 0, st>>>(qb, kb, (const __nv_bfloat16*)v, idx, nsel, pr.B,

@@ -25,7 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 MSA_SELECT, MSA_FWD, MSA_BWD, MSA_DECODE = 0, 1, 2, 3
-MSA_REUSE_INDEX = 1
+MSA_REUSE_INDEX, MSA_DKV_F32 = 1, 2
 _ERR = {0: "ok", -1: "invalid dimensions", -2: "null pointer", -3: "misaligned pointer",
         -4: "workspace too small", -5: "CUDA launch failed", -6: "device wait timed out",
         -7: "device is not sm_100", -8: "tensor map encoding failed",
@@ -42,7 +42,7 @@ class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
                 ("Hp", ctypes.c_int), ("d", ctypes.c_int), ("dp", ctypes.c_int), ("block", ctypes.c_int),
                 ("topk", ctypes.c_int), ("scale", ctypes.c_float), ("window", ctypes.c_int),
-                ("dilation", ctypes.c_int)]
+                ("dilation", ctypes.c_int), ("q_begin", ctypes.c_int)]
 
 
 def _load():
@@ -68,6 +68,8 @@ def _load():
     lib.msa_bwd_ex.restype = I
     lib.msa_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.msa_decode.restype = I
+    lib.msa_f32_to_bf16.argtypes = [P, P, ctypes.c_int64, P]
+    lib.msa_f32_to_bf16.restype = I
     lib.msa_kernel_launches.argtypes = []
     lib.msa_kernel_launches.restype = U64
     for f in ("msa_proxy_select", "msa_fwd", "msa_bwd", "msa_check_status", "msa_diag_umma",
@@ -79,9 +81,9 @@ def _load():
 LIB = _load()
 
 
-def make_dims(B, T, Hq, Hkv, d, dp, topk, scale=0.0, window=1, dilation=1) -> Dims:
+def make_dims(B, T, Hq, Hkv, d, dp, topk, scale=0.0, window=1, dilation=1, q_begin=0) -> Dims:
     return Dims(int(B), int(T), int(Hq), int(Hkv), int(Hkv), int(d), int(dp), 128, int(topk), float(scale),
-                int(window), int(dilation))
+                int(window), int(dilation), int(q_begin))
 
 
 def _p(t):
@@ -132,13 +134,14 @@ def dims_of(q, k, qp, topk, scale=0.0) -> Dims:
     return make_dims(B, T, Hq, Hkv, d, dp, topk, scale)
 
 
-def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False, window=1, dilation=1):
+def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False, window=1, dilation=1, q_begin=0):
     """Index Branch.  Returns (idx, nsel) or (idx, nsel, pooled_scores).
     window/dilation: forced block pattern (own block and the window-1 blocks
-    every `dilation` blocks before it)."""
+    every `dilation` blocks before it).  q_begin: first query row selected
+    (a multiple of 128); earlier rows of the outputs are left unwritten."""
     _bf16(qp, kp)
     B, T, Hp, dp = qp.shape
-    dims = make_dims(B, T, Hp, Hp, 64, dp, topk, window=window, dilation=dilation)
+    dims = make_dims(B, T, Hp, Hp, 64, dp, topk, window=window, dilation=dilation, q_begin=q_begin)
     idx = torch.empty((B, Hp, T, topk), dtype=torch.int32, device=qp.device)
     nsel = torch.empty((B, Hp, T), dtype=torch.int32, device=qp.device)
     nblk = (T + 127) // 128
@@ -152,12 +155,14 @@ def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False, 
     return (idx, nsel, pool) if pooled else (idx, nsel)
 
 
-def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None, reuse_index=False):
-    """Main Branch forward.  Returns (o bf16 [B,T,Hq,d], lse fp32 [B,Hq,T])."""
+def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None, reuse_index=False,
+        q_begin=0):
+    """Main Branch forward.  Returns (o bf16 [B,T,Hq,d], lse fp32 [B,Hq,T]).
+    q_begin: first query row computed; earlier rows of o, lse are unwritten."""
     _bf16(q, k, v)
     B, T, Hq, d = q.shape
     topk = idx.shape[3]
-    dims = make_dims(B, T, Hq, k.shape[2], d, 64, topk, scale)
+    dims = make_dims(B, T, Hq, k.shape[2], d, 64, topk, scale, q_begin=q_begin)
     if out is None:
         o = torch.empty_like(q)
         lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
@@ -173,26 +178,42 @@ def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=No
 
 
 def bwd(q, k, v, o, dout, lse, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None,
-        reuse_index=False):
+        reuse_index=False, q_begin=0, dkv_f32=False):
     """Main Branch backward.  Returns (dq, dk, dv), bf16.  reuse_index: ``ws``
     already holds the inverse index of these idx/nsel from an earlier call on
-    the same workspace (e.g. the forward of the same step)."""
+    the same workspace (e.g. the forward of the same step).  q_begin: first
+    query row computed (dq rows before it are unwritten; dk, dv hold the
+    contributions of the computed rows only).  dkv_f32: dk, dv are fp32
+    unrounded sums, for adding the partials of several query shards."""
     _bf16(q, k, v, o, dout)
     B, T, Hq, d = q.shape
     topk = idx.shape[3]
-    dims = make_dims(B, T, Hq, k.shape[2], d, 64, topk, scale)
+    dims = make_dims(B, T, Hq, k.shape[2], d, 64, topk, scale, q_begin=q_begin)
     if out is None:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dq = torch.empty_like(q)
+        kv_dtype = torch.float32 if dkv_f32 else torch.bfloat16
+        dk = torch.empty(k.shape, dtype=kv_dtype, device=k.device)
+        dv = torch.empty(v.shape, dtype=kv_dtype, device=v.device)
     else:
         dq, dk, dv = out
+    flags = (MSA_REUSE_INDEX if reuse_index else 0) | (MSA_DKV_F32 if dkv_f32 else 0)
     if ws is None:
         ws = workspace(dims, MSA_BWD, q.device)
     _check(LIB.msa_bwd_ex(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(o), _p(dout), _p(lse), _p(idx),
-                          _p(nsel), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream),
-                          MSA_REUSE_INDEX if reuse_index else 0), "msa_bwd")
+                          _p(nsel), _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(), _stream(stream), flags), "msa_bwd")
     if check:
         _check(check_status(ws, stream), "msa_bwd (device)")
     return dq, dk, dv
+
+
+def f32_to_bf16(src, out=None, stream=None):
+    """bf16 copy of a contiguous fp32 CUDA tensor (numel a multiple of 8),
+    rounded on the device by msa_f32_to_bf16."""
+    if src.dtype != torch.float32 or not src.is_cuda or not src.is_contiguous():
+        raise ValueError("expected a contiguous CUDA fp32 tensor")
+    dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device) if out is None else out
+    _check(LIB.msa_f32_to_bf16(_p(src), _p(dst), src.numel(), _stream(stream)), "msa_f32_to_bf16")
+    return dst
 
 
 class MSAAttention(torch.autograd.Function):

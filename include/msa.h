@@ -62,7 +62,21 @@ typedef struct msa_dims {
     float scale;/* softmax scale of the Main Branch; 0 -> 1/sqrt(d)       */
     int window; /* forced blocks per query (own block included); 0 -> 1  */
     int dilation;/* stride between forced blocks; 0 -> 1                 */
+    int q_begin;/* first query row computed: a multiple of 128 in [0, T]; 0 = all */
 } msa_dims;
+
+/*
+ * q_begin (context-parallel shards).  Queries before q_begin are neither
+ * scored, selected nor attended: msa_proxy_select writes idx/nsel (and
+ * pooled_dbg) rows q_begin .. T-1 only, msa_fwd writes those rows of o and lse only, msa_bwd
+ * writes those rows of dq only, and its dk/dv hold the contributions of those
+ * query rows alone -- a partial sum over the keys 0 .. T-1, which the shards
+ * of one sequence add up.  Rows before q_begin of q, qp, dout, o and lse are
+ * not read.  A rank owning query rows [r0, r1) of a sequence passes T = r1,
+ * q_begin = r0, its rows in place and the keys 0 .. r1-1 (the causal prefix
+ * its queries can see).  q_begin = T computes no row (msa_bwd then writes
+ * zero dk/dv).  Decode requires q_begin = 0.
+ */
 
 enum msa_status {
     MSA_OK = 0,
@@ -196,12 +210,20 @@ MSA_API int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q,
  * Reusing an index built from different idx is undefined.  flags = 0 is
  * msa_fwd / msa_bwd.
  */
-enum msa_flags { MSA_REUSE_INDEX = 1 };
+enum msa_flags { MSA_REUSE_INDEX = 1, MSA_DKV_F32 = 2 };
+/* MSA_DKV_F32 (msa_bwd_ex): dk and dv are fp32 [B][T][Hkv][d] and receive the
+ * unrounded sums, so that partial gradients of several query shards can be
+ * added (a reduce-scatter) before one rounding to bf16 (msa_f32_to_bf16). */
 MSA_API int msa_fwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v, const int32_t* idx,
                        const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes, void* stream, int flags);
 MSA_API int msa_bwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v, const void* o,
                        const void* dout, const float* lse, const int32_t* idx, const int32_t* nsel, void* dq,
                        void* dk, void* dv, void* ws, size_t ws_bytes, void* stream, int flags);
+
+/* dst[i] = bf16(src[i]) (round to nearest even) for i < n: fp32 -> bf16 on
+ * the device.  n must be a multiple of 8; both pointers device, 16-byte
+ * aligned.  Used to round partial gradients once they have been summed. */
+MSA_API int msa_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream);
 
 /* Synchronises `stream`, then reads the status word a previous call left in
  * `ws`: MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INDEX.  `code` (nullable)

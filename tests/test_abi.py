@@ -87,7 +87,8 @@ def test_workspace_sizes(lib):
 
 @pytest.mark.parametrize("bad", [dict(d=96), dict(dp=12), dict(dp=72), dict(topk=0), dict(topk=129),
                                  dict(Hq=6, Hkv=4), dict(Hq=12, Hkv=4), dict(T=-1), dict(T=(1 << 20) + 1),
-                                 dict(window=5), dict(window=-1), dict(dilation=-2)])
+                                 dict(window=5), dict(window=-1), dict(dilation=-2),
+                                 dict(q_begin=64), dict(q_begin=-128), dict(q_begin=1152)])
 def test_invalid_dims_rejected(lib, bad):
     d = dims(lib, **bad)
     assert lib.workspace_size(d, lib.MSA_FWD) == 0
@@ -149,3 +150,39 @@ def test_no_gpu_reports_device_error(lib):
     raw, ws = aligned_buffer(256)
     P = 4096
     assert lib.LIB.msa_proxy_select(ctypes.byref(d), P, P, P, P, None, ws, 256, None) == -7
+
+
+def test_q_begin_fields(lib):
+    """q_begin: a block boundary inside [0, T]; the workspaces keep their
+    full-sequence size (the shard's rows sit in place in [0, T))."""
+    full = lib.workspace_size(dims(lib), lib.MSA_FWD)
+    for qb in (0, 128, 896, 1024):
+        assert lib.workspace_size(dims(lib, q_begin=qb), lib.MSA_FWD) == full
+    # ragged T: the last block boundary below T is valid, T itself too
+    assert lib.workspace_size(dims(lib, T=1000, q_begin=896), lib.MSA_SELECT) == 256
+    # decode has one query per sequence: no shard start
+    assert lib.workspace_size(dims(lib, q_begin=128), lib.MSA_DECODE) == 0
+
+
+def test_q_begin_at_t_is_a_no_op(lib):
+    """Nothing to compute: selection and forward return at once, without
+    looking at the tensor pointers or the device."""
+    raw, ws = aligned_buffer(1 << 20)
+    d = dims(lib, q_begin=1024)
+    need = lib.workspace_size(d, lib.MSA_FWD)
+    assert lib.LIB.msa_fwd(ctypes.byref(d), None, None, None, None, None, None, None, ws, need, None) == 0
+    assert lib.LIB.msa_proxy_select(ctypes.byref(d), None, None, None, None, None, ws, 256, None) == 0
+    # the backward zeroes dk, dv: it needs them (and a device)
+    nb = lib.workspace_size(d, lib.MSA_BWD)
+    assert lib.LIB.msa_bwd(ctypes.byref(d), None, None, None, None, None, None, None, None, None, None, None,
+                           ws, nb, None) == -2
+
+
+def test_f32_to_bf16_argument_checks(lib):
+    P = 4096
+    assert lib.LIB.msa_f32_to_bf16(P, P, 12, None) == -1      # not a multiple of 8
+    assert lib.LIB.msa_f32_to_bf16(P, P, -8, None) == -1
+    assert lib.LIB.msa_f32_to_bf16(None, None, 0, None) == 0  # empty
+    assert lib.LIB.msa_f32_to_bf16(None, P, 8, None) == -2
+    assert lib.LIB.msa_f32_to_bf16(P + 4, P, 8, None) == -3
+

@@ -1,0 +1,161 @@
+"""Context-parallel MSA (one sequence split by rows over the ranks), host
+side, on CPU: the shard split, and a whole step over two and three gloo
+ranks -- all-gather of the key side, per-rank selection, forward and
+backward of its own query rows (q_begin), reduce-scatter of the fp32 partial
+dK/dV -- against the oracle run on the unsplit sequence.
+
+The per-rank attention here is the oracle behind the library's call
+signatures (a test stand-in: on GPUs the same orchestration calls the CUDA
+library, checked in test_gpu_cp.py); what these tests pin is the
+decomposition and the collectives, with a real process group.
+"""
+import os
+import socket
+import sys
+import types
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_attention_09_b200 import cp  # noqa: E402
+from block_sparse_attention_09_b200.inputs import Config, make_inputs  # noqa: E402
+
+
+class OracleOps:
+    """The oracle behind the library's Python call signatures (CPU tensors).
+    Rows before q_begin are neither selected nor computed, as in the library."""
+
+    import oracle as O
+
+    @staticmethod
+    def make_dims(B, T, Hq, Hkv, d, dp, topk, scale=0.0, window=1, dilation=1, q_begin=0):
+        return types.SimpleNamespace(B=B, T=T, Hq=Hq, Hkv=Hkv, d=d, dp=dp, topk=topk, q_begin=q_begin)
+
+    @staticmethod
+    def step_workspace(dims, device):
+        return {}
+
+    @classmethod
+    def _m(cls, B, T, Hq, Hkv, d, dp, topk):
+        return cls.O.Dims(B=B, T=T, Hq=Hq, Hkv=Hkv, d=d, dp=dp, topk=topk)
+
+    @classmethod
+    def proxy_select(cls, qp, kp, topk, q_begin=0):
+        B, T, Hp, dp = qp.shape
+        m = cls._m(B, T, Hp, Hp, 64, dp, topk)
+        rows = [(b * Hp + g) * T + i for b in range(B) for g in range(Hp) for i in range(q_begin, T)]
+        idx, nsel, _ = cls.O.select(m, qp.float().numpy(), kp.float().numpy(), rows=rows)
+        return torch.from_numpy(idx), torch.from_numpy(nsel)
+
+    @classmethod
+    def fwd(cls, q, k, v, idx, nsel, scale=0.0, ws=None, q_begin=0):
+        B, T, Hq, d = q.shape
+        m = cls._m(B, T, Hq, k.shape[2], d, 64, idx.shape[3])
+        rows = [(b * Hq + h) * T + i for b in range(B) for h in range(Hq) for i in range(q_begin, T)]
+        o, lse = cls.O.fwd(m, q.float().numpy(), k.float().numpy(), v.float().numpy(), idx.numpy(), nsel.numpy(),
+                           rows=rows)
+        return torch.from_numpy(o).to(torch.bfloat16), torch.from_numpy(lse).float()
+
+    @classmethod
+    def bwd(cls, q, k, v, o, dout, lse, idx, nsel, scale=0.0, ws=None, reuse_index=False, q_begin=0,
+            dkv_f32=False):
+        B, T, Hq, d = q.shape
+        m = cls._m(B, T, Hq, k.shape[2], d, 64, idx.shape[3])
+        rows = [(b * Hq + h) * T + i for b in range(B) for h in range(Hq) for i in range(q_begin, T)]
+        x = [t.float().numpy() for t in (q, k, v, dout)]
+        dq, D = cls.O.bwd_dq(m, *x, o.float().numpy().astype(np.float64), lse.numpy().astype(np.float64),
+                             idx.numpy(), nsel.numpy(), rows=rows)
+        # rows before q_begin selected nothing, so every block's selecting
+        # queries are this shard's: the partial dK, dV of its rows
+        dk, dv = cls.O.bwd_dkdv(m, *x, lse.numpy().astype(np.float64), D, idx.numpy(), nsel.numpy())
+        kv = torch.float32 if dkv_f32 else torch.bfloat16
+        return torch.from_numpy(dq).to(torch.bfloat16), torch.from_numpy(dk).to(kv), torch.from_numpy(dv).to(kv)
+
+    @staticmethod
+    def f32_to_bf16(x):
+        return x.to(torch.bfloat16)
+
+
+def test_shard_bounds_cover_the_sequence():
+    for T in (1, 127, 128, 640, 1000, 4096, 131072 + 77):
+        for world in (1, 2, 3, 4, 8):
+            b = [cp.shard_bounds(T, world, r) for r in range(world)]
+            assert b[0][0] == 0 and b[-1][1] == T
+            for (a0, a1), (c0, c1) in zip(b, b[1:]):
+                assert a1 == c0                      # contiguous
+            for r0, r1 in b:
+                assert r0 % 128 == 0 and r0 <= r1    # block aligned
+            nb = [(r1 - r0 + 127) // 128 for r0, r1 in b]
+            assert max(nb) - min(nb) <= 1            # balanced by whole blocks
+
+
+CFG = Config("cp", B=1, T=1000, Hq=4, Hkv=2, d=64, dp=32, topk=3)
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    from datetime import timedelta
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=120))
+    try:
+        x = make_inputs(CFG, seed=3, exact_proxy=True)
+        r0, r1 = cp.shard_bounds(CFG.T, world, rank)
+        mine = {k: t[:, r0:r1].contiguous() for k, t in x.items()}
+        o, lse, dq, dk, dv = cp.step(mine["q"], mine["k"], mine["v"], mine["dout"], mine["qp"], mine["kp"],
+                                     CFG.topk, CFG.T, ops=OracleOps)
+        torch.save(dict(r0=r0, r1=r1, o=o, lse=lse, dq=dq, dk=dk, dv=dv), os.path.join(out_dir, f"rank{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_cp_step_matches_the_unsplit_sequence(tmp_path, oracle_mod, world):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, str(tmp_path))) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+        assert p.exitcode == 0, f"rank exited with {p.exitcode}"
+    O = oracle_mod
+    x = {k: t.float().numpy() for k, t in make_inputs(CFG, seed=3, exact_proxy=True).items()}
+    m = O.Dims(B=CFG.B, T=CFG.T, Hq=CFG.Hq, Hkv=CFG.Hkv, d=CFG.d, dp=CFG.dp, topk=CFG.topk)
+    # the unsplit sequence, with the backward's D taken from the bf16-stored O
+    # as the library (and the stand-in) does
+    idx, nsel, _ = O.select(m, x["qp"], x["kp"])
+    o, lse = O.fwd(m, x["q"], x["k"], x["v"], idx, nsel)
+    o16 = torch.from_numpy(o).to(torch.bfloat16).float().numpy().astype(np.float64)
+    dq, D = O.bwd_dq(m, x["q"], x["k"], x["v"], x["dout"], o16, lse, idx, nsel)
+    dk, dv = O.bwd_dkdv(m, x["q"], x["k"], x["v"], x["dout"], lse, D, idx, nsel)
+    ref = dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv)
+    covered = 0
+    for r in range(world):
+        got = torch.load(tmp_path / f"rank{r}.pt")
+        r0, r1 = got["r0"], got["r1"]
+        covered += r1 - r0
+        sl = slice(r0, r1)
+        # bf16 outputs: within the rounding of one bf16 store (dK/dV: two
+        # shards' fp32 partials added before the one rounding)
+        for name, g, rf in (("o", got["o"], ref["o"][:, sl]), ("dq", got["dq"], ref["dq"][:, sl]),
+                            ("dk", got["dk"], ref["dk"][:, sl]), ("dv", got["dv"], ref["dv"][:, sl])):
+            err = np.abs(g.float().numpy() - rf)
+            assert (err <= 1e-6 + 2.0 ** -8 * np.abs(rf)).all(), (name, r, float(err.max()))
+        assert np.allclose(got["lse"].numpy(), ref["lse"][:, :, sl], rtol=1e-6, atol=1e-5)
+    assert covered == CFG.T
