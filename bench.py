@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--decode", action="store_true",
                     help="time msa_decode (one new token per sequence against full-length caches) instead")
     ap.add_argument("--decode-batch", type=int, default=16, help="sequences per decode step")
+    ap.add_argument("--cp", action="store_true",
+                    help="context parallel: one sequence of the workload split by rows over the ranks "
+                         "(key-side all-gather, dK/dV reduce-scatter); strong scaling")
     ap.add_argument("--window", type=int, default=1, help="forced blocks per query (own block included)")
     ap.add_argument("--dilation", type=int, default=1, help="stride between forced blocks")
     ap.add_argument("--bias", default=None, choices=["none", "group", "recency"],
@@ -324,6 +327,84 @@ def run_decode(args, cfg, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_cp(args, cfg, rank, local, world):
+    """Context-parallel step: the workload's sequence split into equal 128-row
+    shards over the ranks (block_sparse_attention_09_b200.cp): all-gather of
+    k, v, kp, each rank's selection, forward and backward of its own query
+    rows, reduce-scatter of the fp32 partial dK/dV.  The work is fixed as the
+    ranks grow (strong scaling); value = FLOPs of the whole sequence's step /
+    the slowest rank's time."""
+    import torch
+    import torch.distributed as dist
+    from block_sparse_attention_09_b200 import cp, msa
+    from block_sparse_attention_09_b200.inputs import make_inputs
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
+    r0, r1 = cp.shard_bounds(cfg.T, world, rank)
+    host = make_inputs(cfg, seed=0)   # the same sequence on every rank; each keeps its rows
+    d = {k: v[:, r0:r1].contiguous().to(dev) for k, v in host.items()}
+    del host
+
+    def step():
+        return cp.step(d["q"], d["k"], d["v"], d["dout"], d["qp"], d["kp"], cfg.topk, cfg.T, return_selection=True)
+
+    out = step()
+    nsel = out[6]
+    # selected-key pairs of this rank's rows, summed over the ranks
+    i = torch.arange(r0, r1, device=dev, dtype=torch.int64)
+    pairs = (BLOCK * (nsel.to(torch.int64) - 1) + ((i % BLOCK) + 1).view(1, 1, -1)).sum().double()
+    if world > 1:
+        dist.all_reduce(pairs)
+    f_proxy, f_fwd, f_bwd = flops_from_nsel(cfg, {"pairs": float(pairs.item())})
+    f_step = f_proxy + f_fwd + f_bwd
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    l0 = msa.kernel_launches()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b_.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = a.elapsed_time(b_) / args.steps
+    launches = msa.kernel_launches() - l0
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks, src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    tflops = f_step / (ms * 1e-3) / 1e12
+    line = {"metric": METRIC + " (context parallel)", "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) bf16 inputs" + (", planted local-recency proxy bias" if cfg.bias == "recency" else ""),
+            "config": {"workload": workload_name(cfg) + f", rows split over {world} ranks",
+                       "B": cfg.B, "T": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "dp": cfg.dp,
+                       "topk": cfg.topk, "parallelism": f"cp{world}",
+                       "l2": "inputs larger than L2, no flush"},
+            "tokens_per_s": cfg.B * cfg.T / (ms * 1e-3),
+            "flops_per_step": {"proxy": f_proxy, "fwd": f_fwd, "bwd": f_bwd},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "traffic": None,
+                         "peak_source": f"{src} bf16 sustained (whole step, collectives included)"},
+            "cpu_baseline": None, "e2e": None,
+            "gpu_launches": launches}
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     args = parse()
@@ -340,6 +421,9 @@ def main():
         return
     if args.decode:
         run_decode(args, cfg, rank, local)
+        return
+    if args.cp:
+        run_cp(args, cfg, rank, local, world)
         return
 
     import torch

@@ -94,15 +94,23 @@ def local_step(q, k_pre, v_pre, dout, qp, kp_pre, topk, r0, ops, scale=0.0):
     return (o[:, r0:].contiguous(), lse[:, :, r0:].contiguous(), dq[:, r0:].contiguous(), dk, dv, idx, nsel)
 
 
-def step(q, k, v, dout, qp, kp, topk, T, group=None, ops=None, scale=0.0):
+def step(q, k, v, dout, qp, kp, topk, T, group=None, ops=None, scale=0.0, return_selection=False):
     """One context-parallel MSA training step.  Every rank passes its own rows
     [r0, r1) = shard_bounds(T, world, rank) of q, k, v, dout, qp, kp
     ([B, r1-r0, H, d]).  Returns this rank's rows of o, lse ([B, Hq, r1-r0]),
-    dq, and of dk, dv summed over every rank's queries."""
+    dq, and of dk, dv summed over every rank's queries (and, with
+    return_selection, its rows' idx [B, Hp, r1-r0, topk] and nsel).  Without
+    an initialised process group the step runs as the only rank."""
     if ops is None:
         from . import msa as ops
-    world = dist.get_world_size(group)
-    rank = dist.get_rank(group)
+    if dist.is_available() and dist.is_initialized():
+        world, rank = dist.get_world_size(group), dist.get_rank(group)
+    else:
+        world, rank = 1, 0
+    if world == 1:
+        o, lse, dq, dk_part, dv_part, idx, nsel = local_step(q, k, v, dout, qp, kp, topk, 0, ops, scale)
+        out = (o, lse, dq, ops.f32_to_bf16(dk_part), ops.f32_to_bf16(dv_part))
+        return out + (idx, nsel) if return_selection else out
     bounds = [shard_bounds(T, world, j) for j in range(world)]
     r0, r1 = bounds[rank]
     assert q.shape[1] == r1 - r0
@@ -112,8 +120,10 @@ def step(q, k, v, dout, qp, kp, topk, T, group=None, ops=None, scale=0.0):
     kp_all = _gather_rows(kp, group, world, bounds)
     k_pre, v_pre, kp_pre = (x[:, :r1].contiguous() for x in (k_all, v_all, kp_all))
     # 2. this rank's queries
-    o, lse, dq, dk_part, dv_part, _, _ = local_step(q, k_pre, v_pre, dout, qp, kp_pre, topk, r0, ops, scale)
+    o, lse, dq, dk_part, dv_part, idx, nsel = local_step(q, k_pre, v_pre, dout, qp, kp_pre, topk, r0, ops, scale)
     # 3. gradients of this rank's keys, summed over all ranks, rounded once
     dk = ops.f32_to_bf16(_reduce_scatter_rows(dk_part, group, world, rank, bounds))
     dv = ops.f32_to_bf16(_reduce_scatter_rows(dv_part, group, world, rank, bounds))
+    if return_selection:
+        return o, lse, dq, dk, dv, idx[:, :, r0:].contiguous(), nsel[:, :, r0:].contiguous()
     return o, lse, dq, dk, dv

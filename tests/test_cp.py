@@ -159,3 +159,19 @@ def test_cp_step_matches_the_unsplit_sequence(tmp_path, oracle_mod, world):
             assert (err <= 1e-6 + 2.0 ** -8 * np.abs(rf)).all(), (name, r, float(err.max()))
         assert np.allclose(got["lse"].numpy(), ref["lse"][:, :, sl], rtol=1e-6, atol=1e-5)
     assert covered == CFG.T
+
+
+def test_single_rank_without_a_process_group(oracle_mod):
+    """No process group: the step is the whole sequence on one rank (q_begin
+    0, fp32 gradients rounded once), equal to the unsplit oracle run."""
+    O = oracle_mod
+    x = make_inputs(CFG, seed=4, exact_proxy=True)
+    o, lse, dq, dk, dv, idx, nsel = cp.step(x["q"], x["k"], x["v"], x["dout"], x["qp"], x["kp"], CFG.topk, CFG.T,
+                                            ops=OracleOps, return_selection=True)
+    xf = {k: t.float().numpy() for k, t in x.items()}
+    m = O.Dims(B=CFG.B, T=CFG.T, Hq=CFG.Hq, Hkv=CFG.Hkv, d=CFG.d, dp=CFG.dp, topk=CFG.topk)
+    ref = O.full(m, xf["qp"], xf["kp"], xf["q"], xf["k"], xf["v"], xf["dout"])
+    assert np.array_equal(idx.numpy(), ref["idx"]) and np.array_equal(nsel.numpy(), ref["nsel"])
+    err = np.abs(o.float().numpy() - ref["o"])
+    assert (err <= 1e-6 + 2.0 ** -8 * np.abs(ref["o"])).all()
+    assert np.allclose(lse.numpy(), ref["lse"], rtol=1e-6, atol=1e-5)
