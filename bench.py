@@ -82,9 +82,11 @@ def flops_from_nsel(cfg, nsel_counts):
     return f_proxy, f_fwd, f_bwd
 
 
-def pair_count(cfg, nsel):
+def pair_count(cfg, nsel, r0=0):
+    """Selected (query, key) pairs of the rows r0 .. r0 + nsel.shape[2] - 1
+    whose selection sizes nsel [B, Hp, rows] holds."""
     import torch
-    i = torch.arange(cfg.T, device=nsel.device, dtype=torch.int64)
+    i = torch.arange(r0, r0 + nsel.shape[2], device=nsel.device, dtype=torch.int64)
     own = (i % BLOCK) + 1
     pairs = BLOCK * (nsel.to(torch.int64) - 1) + own.view(1, 1, -1)
     return {"pairs": float(pairs.sum().item())}
@@ -354,8 +356,7 @@ def run_cp(args, cfg, rank, local, world):
     out = step()
     nsel = out[6]
     # selected-key pairs of this rank's rows, summed over the ranks
-    i = torch.arange(r0, r1, device=dev, dtype=torch.int64)
-    pairs = (BLOCK * (nsel.to(torch.int64) - 1) + ((i % BLOCK) + 1).view(1, 1, -1)).sum().double()
+    pairs = torch.tensor([pair_count(cfg, nsel, r0)["pairs"]], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(pairs)
     f_proxy, f_fwd, f_bwd = flops_from_nsel(cfg, {"pairs": float(pairs.item())})

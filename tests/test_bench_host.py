@@ -39,6 +39,21 @@ def test_flop_model_counts_the_selected_pairs():
     assert f_proxy == 2.0 * cfg.dp * scored * cfg.B * cfg.Hkv
 
 
+def test_pair_count_of_row_shards_adds_up():
+    """The context-parallel bench counts each rank's rows from its own row
+    offset: the shards' counts add up to the whole sequence's."""
+    cfg = Config("shards", B=2, T=1000, Hq=4, Hkv=2, d=64, dp=32, topk=3)
+    g = torch.Generator().manual_seed(5)
+    i = torch.arange(cfg.T)
+    nsel = torch.minimum(torch.randint(1, cfg.topk + 1, (cfg.B, cfg.Hkv, cfg.T), generator=g), i // 128 + 1)
+    whole = bench.pair_count(cfg, nsel)["pairs"]
+    brute = sum(128 * (int(nsel[b, h, r]) - 1) + r % 128 + 1
+                for b in range(cfg.B) for h in range(cfg.Hkv) for r in range(cfg.T))
+    assert whole == brute
+    parts = sum(bench.pair_count(cfg, nsel[:, :, r0:r1], r0)["pairs"] for r0, r1 in ((0, 256), (256, 640), (640, 1000)))
+    assert parts == whole
+
+
 def test_recorded_traffic_needs_unchanged_sources(tmp_path, monkeypatch):
     csrc = tmp_path / "block_sparse_attention_09_b200" / "csrc"
     csrc.mkdir(parents=True)
