@@ -21,6 +21,9 @@ training, paragraphs 1-4):
 * ``bwd_dq``  -- dQ and D = dO . O per query row.
 * ``bwd_dkdv``-- dK, dV per KV block, summed over every selecting query and
   every head of the group.
+
+``proxy_grad`` (numpy) holds a proxy-head training loss and its gradient; the
+pages do not describe one, so it is a reading, and its parity is unpinned.
 """
 from __future__ import annotations
 
