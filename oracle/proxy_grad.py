@@ -15,9 +15,10 @@ attention.  The reading written out here follows that: per query row
     q_i    = softmax over n in S_i of z_i(n),
     loss   = sum_i KL(p_i || q_i) = sum_i sum_n p_i(n) (log p_i(n) - log q_i(n)),
 
-and the gradient d loss / d z_i(n) = q_i(n) - p_i(n) goes through the
-max-pool to its argmax key j* (the lowest j on ties): dqp_i += (q - p) kp_j*,
-dkp_j* += (q - p) qp_i.  The selection itself is fixed (passed in): top-k is
+and the gradient d loss / d z_i(n) = q_i(n) sum_m p_i(m) - p_i(n) (which is
+q_i(n) - p_i(n) when p_i sums to one) goes through the
+max-pool to its argmax key j* (the lowest j on ties): dqp_i += dz kp_j*,
+dkp_j* += dz qp_i.  The selection itself is fixed (passed in): top-k is
 not differentiable.
 
 Plain numpy in float64, one row at a time.  The tests pin it by finite
@@ -83,7 +84,7 @@ def loss_and_grad(m, qp, kp, q, k, lse, idx, nsel, rows=None):
         lq = z - zmax - np.log(np.exp(z - zmax).sum())   # log q
         pos = p > 0
         total += float((p[pos] * (np.log(p[pos]) - lq[pos])).sum())
-        dz = np.exp(lq) - p
+        dz = np.exp(lq) * p.sum() - p   # exact derivative, whatever the mass of p
         qv = qp[b, i, g].astype(np.float64)
         for s in range(len(z)):
             j = int(arg[s])
