@@ -51,14 +51,20 @@ def parse():
     ap.add_argument("--dilation", type=int, default=1, help="stride between forced blocks")
     ap.add_argument("--bias", default=None, choices=["none", "group", "recency"],
                     help="override the workload's proxy-input structure (profiling variants)")
+    ap.add_argument("--outliers", type=int, default=0,
+                    help="large-norm (x8) key rows per (batch, group): the attention-sink-like variant")
+    ap.add_argument("--groups", type=int, default=0,
+                    help="run only this many of the workload's KV groups (same per-group shape; profiling "
+                         "captures scale their counters by the group ratio)")
     return ap.parse_args()
 
 
 def workload_name(cfg, window=1, dilation=1):
     bias = {"none": "", "group": ", per-group low-rank proxy bias", "recency": ", planted local-recency proxy bias"}
     pattern = f", forced window {window} blocks at dilation {dilation}" if window > 1 else ""
+    outl = f", {cfg.k_outliers} large-norm (x8) keys per group" if cfg.k_outliers else ""
     return (f"MSA {cfg.name}: B={cfg.B} T={cfg.T} Hq={cfg.Hq} Hkv={cfg.Hkv} d={cfg.d} dp={cfg.dp} "
-            f"topk={cfg.topk} (own block incl.), causal, fwd+bwd{bias[cfg.bias]}{pattern}")
+            f"topk={cfg.topk} (own block incl.), causal, fwd+bwd{bias[cfg.bias]}{pattern}{outl}")
 
 
 # ---------------------------------------------------------------- FLOP model
@@ -144,26 +150,36 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary of this
-    workload, or None when there is none or the kernel's sources have changed
-    since it was captured (the summary records their sha256)."""
+def sources_sha256(names):
+    """sha256 over the named files under the package's csrc/, in order (the
+    key a committed traffic record was taken with); None if one is missing."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"dram_msa_{workload}.md")
+    csrc = os.path.join(ROOT, "block_sparse_attention_09_b200", "csrc")
+    h = hashlib.sha256()
+    for name in names:
+        fp = os.path.join(csrc, name)
+        if not os.path.exists(fp):
+            return None
+        with open(fp, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    record profiles/traffic.json (the capture's bytes times its stated scale
+    to the full launch), or None when there is none or the kernel's sources
+    have changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    csrc = os.path.join(ROOT, "block_sparse_attention_09_b200", "csrc")
-    for line in open(path):
-        parts = line.split()
-        if len(parts) == 5 and parts[0] == "traffic" and parts[1] == kernel:
-            h = hashlib.sha256()
-            for name in parts[3].split(","):
-                fp = os.path.join(csrc, name)
-                if not os.path.exists(fp):
-                    return None
-                with open(fp, "rb") as f:
-                    h.update(f.read())
-            return float(parts[2]) if h.hexdigest() == parts[4] else None
+    with open(path) as f:
+        rec = json.load(f)
+    for r in rec.get("records", []):
+        if r.get("kernel") == kernel and r.get("workload") == workload:
+            if sources_sha256(r["sources"]) != r["sources_sha256"]:
+                return None
+            return float(r["bytes_per_launch_captured"]) * float(r["scale_to_full"])
     return None
 
 
@@ -413,6 +429,10 @@ def main():
     cfg = CONFIGS[args.config]
     if args.bias is not None:
         cfg = cfg.with_(bias=args.bias)
+    if args.outliers:
+        cfg = cfg.with_(k_outliers=args.outliers)
+    if args.groups:
+        cfg = cfg.with_(name=f"{cfg.name}-g{args.groups}", Hkv=args.groups, Hq=args.groups * cfg.G)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -472,6 +492,7 @@ def main():
     idx, nsel = msa.proxy_select(d["qp"], d["kp"], cfg.topk, ws=ws_sel, window=args.window,
                                  dilation=args.dilation, check=True)
     msa.fwd(d["q"], d["k"], d["v"], idx, nsel, ws=ws_fwd, out=(o, lse), check=True)
+    fallback = msa.fallback_rows(ws_fwd)   # rows the forward redid with its exact two-pass softmax
     msa.bwd(d["q"], d["k"], d["v"], o, d["dout"], lse, idx, nsel, ws=ws_bwd, out=(dq, dk, dv), reuse_index=True,
             check=True)
     f_proxy, f_fwd, f_bwd = flops_from_nsel(cfg, pair_count(cfg, nsel))
@@ -658,6 +679,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
+        "fallback_rows": fallback,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

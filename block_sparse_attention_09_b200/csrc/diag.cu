@@ -12,8 +12,7 @@ namespace msa {
 namespace {
 
 // mode: 0 A,B K-major | 1 A K-major, B MN-major | 2 A,B MN-major |
-//       3 A TMEM, B MN-major | 4 A TMEM, B K-major.  +8: MN-major descriptors
-//       with the two byte offsets exchanged (to check that convention).
+//       3 A TMEM, B MN-major | 4 A TMEM, B K-major.
 __global__ void __launch_bounds__(128, 1) diag_umma_kernel(int mode, int N, int K,
                                                            const __nv_bfloat16* __restrict__ A,
                                                            const __nv_bfloat16* __restrict__ B,
@@ -27,8 +26,6 @@ __global__ void __launch_bounds__(128, 1) diag_umma_kernel(int mode, int N, int 
     uint32_t* tmem_hold = (uint32_t*)(bar + 1);
     volatile uint32_t* abort_flag = tmem_hold + 1;
     const int t = threadIdx.x, warp = t >> 5;
-    const bool swap = (mode & 8) != 0;
-    mode &= 7;
     const bool a_tmem = mode >= 3;
     const bool a_mn = mode == 2;
     const bool b_mn = mode == 1 || mode == 2 || mode == 3;
@@ -98,15 +95,13 @@ __global__ void __launch_bounds__(128, 1) diag_umma_kernel(int mode, int N, int 
         for (int kk = 0; kk < K / 16; ++kk) {
             uint64_t bd;
             if (!b_mn) bd = desc_kmajor(ba, (uint32_t)N, kk * 16);
-            else if (!swap) bd = desc_mnmajor(ba, (uint32_t)K, kk * 16);
-            else bd = umma_desc(ba + kk * 16 * 128, 1024u, (uint32_t)K * 128u);
+            else bd = desc_mnmajor(ba, (uint32_t)K, kk * 16);
             if (a_tmem) {
                 umma_ts(tmem, tmem + 128u + kk * 8, bd, idesc, kk > 0 ? 1u : 0u);
             } else {
                 uint64_t ad;
                 if (!a_mn) ad = desc_kmajor(aa, 128, kk * 16);
-                else if (!swap) ad = desc_mnmajor(aa, (uint32_t)K, kk * 16);
-                else ad = umma_desc(aa + kk * 16 * 128, 1024u, (uint32_t)K * 128u);
+                else ad = desc_mnmajor(aa, (uint32_t)K, kk * 16);
                 umma_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
             }
         }

@@ -28,24 +28,29 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_fwd_scratch[kNoAllocScratchBytes];
 
-struct ScratchSlot {
-    std::once_flag once;
-    void* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
-ScratchSlot g_slots[kMaxDevices];
+std::mutex g_slot_mutex;
+void* g_slot_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device, with that device current.
+// once per device, with that device current.  A failed look-up (the module
+// holding the array could not be loaded, e.g. out of device memory) is not
+// remembered: the next call tries again, and the runtime's error state is
+// cleared so that it cannot surface in an unrelated later call.
 int scratch_on_current_device(void** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MSA_ERR_DEVICE;
-    ScratchSlot& s = g_slots[dev];
-    std::call_once(s.once, [&s] { s.err = cudaGetSymbolAddress(&s.ptr, g_fwd_scratch); });
-    if (s.err != cudaSuccess || s.ptr == nullptr) return MSA_ERR_LAUNCH;
-    *out = s.ptr;
+    std::lock_guard<std::mutex> lock(g_slot_mutex);
+    if (g_slot_ptr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_fwd_scratch) != cudaSuccess || ptr == nullptr) {
+            (void)cudaGetLastError();
+            return MSA_ERR_LAUNCH;
+        }
+        g_slot_ptr[dev] = ptr;
+    }
+    *out = g_slot_ptr[dev];
     return MSA_OK;
 }
 

@@ -27,11 +27,10 @@ WsLayout ws_layout(const Problem& p, int which)
         L.tok = take(BH * (size_t)p.T * p.topk * 4);
     }
     if (which == MSA_FWD) {
-        L.qnorm = take(rows * 4);
-        L.kmax = take((size_t)p.B * p.Hkv * 4);
+        L.shift = take(rows * 4);
+        L.kmax = take((size_t)p.B * p.Hkv * p.nblk * 4);
         L.oacc = take(rows * p.d * 4);
         L.lacc = take(rows * 4);
-        L.nflag = take(4);
         L.flags = take(rows * 4);
     }
     if (which == MSA_DECODE) {
@@ -316,6 +315,17 @@ int msa_check_status(const void* ws, void* stream, uint32_t* code)
     return MSA_OK;
 }
 
+int msa_fallback_rows(const void* ws, void* stream, int64_t* rows)
+{
+    if (!ws || !rows) return MSA_ERR_NULL_PTR;
+    uint32_t w = 0;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MSA_ERR_LAUNCH;
+    if (cudaMemcpy(&w, (const uint32_t*)ws + 2, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MSA_ERR_LAUNCH;
+    *rows = (int64_t)w;
+    return MSA_OK;
+}
+
 const char* msa_strerror(int s)
 {
     switch (s) {
@@ -346,7 +356,7 @@ int msa_set_kernel_events(int kernel, void* start, void* stop)
 
 int msa_diag_umma(int mode, int N, int K, const void* A, const void* B, float* D, void* ws, void* stream)
 {
-    if ((mode & 7) > 4 || (N != 64 && N != 128) || (K != 64 && K != 128)) return MSA_ERR_INVALID_DIMS;
+    if (mode < 0 || mode > 4 || (N != 64 && N != 128) || (K != 64 && K != 128)) return MSA_ERR_INVALID_DIMS;
     if (!A || !B || !D || !ws) return MSA_ERR_NULL_PTR;
     if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(ws, 256)) return MSA_ERR_MISALIGNED;
     int rc = check_device();

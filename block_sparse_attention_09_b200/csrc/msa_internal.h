@@ -33,9 +33,9 @@ struct Problem {
 
 // Byte offsets of the workspace regions.
 struct WsLayout {
-    size_t status = 0;                           // 256 B: status word, index-error word
+    size_t status = 0;   // 256 B: [0] timeout code, [1] index error, [2] forward fallback rows
     size_t cnt = 0, tot = 0, ptr = 0, tok = 0;   // block -> query inverse index
-    size_t qnorm = 0, kmax = 0, oacc = 0, lacc = 0, nflag = 0, flags = 0;   // forward
+    size_t shift = 0, kmax = 0, oacc = 0, lacc = 0, flags = 0;   // forward
     size_t dsum = 0, dqacc = 0, dkacc = 0, dvacc = 0;   // backward
     size_t pooled = 0, part = 0;                        // decode
     size_t total = 0;

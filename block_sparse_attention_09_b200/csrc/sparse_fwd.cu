@@ -11,17 +11,27 @@
 // block are gathered from the inverse index in chunks of 128 rows (128/G
 // tokens x the G query heads of the group, head-major: row = hh * 128/G + t)
 // with cp.async into a 3-stage ring.
-// Per chunk:  S = Q K^T (tcgen05, TMEM) -> P = exp(S*scale - bound) written
+// Per chunk:  S = Q K^T (tcgen05, TMEM) -> P = exp2(S*scale*log2e - m_i) written
 // back to TMEM as bf16 -> O_part = P V (tcgen05 with A from TMEM) -> fp32
 // reductions of O_part and of the row sums into global accumulators.
 //
 // Softmax normalisation across the CTAs that share a query row uses a fixed
-// per-row shift instead of a running maximum: the Cauchy-Schwarz bound
-// |scale| * |q_i| * max_j |k_j| is never below any score, so exp(S - bound)
-// cannot overflow and every CTA's partial sums are directly additive.  The
-// finalize pass divides by the row sum and sets L = bound + log(sum).  Rows
-// whose sum underflows (bound far above the true maximum) are listed and
-// recomputed exactly by a fallback kernel with a two-pass softmax.
+// per-row shift m_i instead of a running maximum, so every CTA's partial sums
+// are directly additive.  m_i only has to lie near the row's true maximum
+// score (in log2 units, within what fp32 exponents absorb), and it is
+// bracketed by two values known before any CTA starts:
+//   U_i = |scale| |q_i| max over the row's selected blocks of max |k_j|
+//         (Cauchy-Schwarz: no score of the row is above it), and
+//   S_ii = the score of the query's own key, which every row reads (own
+//         block forced, j = i visible): the row maximum is at least S_ii.
+// With m_i = min(U_i, S_ii + 100) (log2 units) the largest weight
+// exp2(S - m_i) is in [2^-100, 1] unless the row's best score exceeds S_ii
+// by more than 100 (then m_i = S_ii + 100 and weights may grow large).  A
+// single large-norm key therefore no longer loosens the shift of the rows
+// that read it.  The finalize pass divides by the row sum and sets
+// L = (m_i + log2 sum) ln 2.  Rows whose sum is outside [2^-110, 2^100] (or
+// not finite) are listed and recomputed exactly by a fallback kernel with a
+// two-pass softmax.
 #include <math.h>
 
 #include "msa_device.cuh"
@@ -33,19 +43,19 @@ namespace {
 constexpr int kThreads = 448;   // w0 TMA(K,V) | w1 MMA | w2-5 gather | w6-9 softmax | w10-13 O out
 constexpr int kQStages = 3;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kUnderflow = 5.421010862427522e-20f;   // 2^-64: row sums below are redone exactly
+constexpr float kSumLow = 7.703719777548943e-34f;     // 2^-110: row sums outside [kSumLow, kSumHigh]
+constexpr float kSumHigh = 1.2676506002282294e30f;    // 2^100   (or not finite) are redone exactly
+constexpr float kShiftSlack = 100.f;                  // m_i <= S_ii + kShiftSlack (log2 units)
 
 struct FwdParams {
     int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
     int RB, qb0, per_group;   // query blocks per range; first query block; work items per (b, group)
     float c1;        // scale * log2(e)
-    float bound;     // |scale| * log2(e)
     const __nv_bfloat16* q;
     const int32_t* ptr;
     const int32_t* off;
     const int32_t* tok;
-    const float* qn;
-    const float* kmax;
+    const float* shift;   // m_i per [b][h][i], log2 units
     float* oacc;
     float* lacc;
     uint32_t* status;
@@ -200,32 +210,31 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         cp_async_wait<0>();
     } else if (warp < 10) {
-        // ---------------- softmax: P = exp2(S*c1 - bound) ----------------
+        // ---------------- softmax: P = exp2(S*c1 - m_i) ----------------
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
         const int t = r & (p.tpc - 1), hh = r >> (7 - p.lgG), h = g * G + hh;
-        const float kmx = p.kmax[bg];
-        const float* qn_row = p.qn + ((int64_t)b * p.Hq + h) * p.T;
-        // this row's token and |q| are loaded one and two chunks ahead, so the
-        // dependent global loads overlap the previous chunk's work
+        const float* shift_row = p.shift + ((int64_t)b * p.Hq + h) * p.T;
+        // this row's token and shift are loaded one and two chunks ahead, so
+        // the dependent global loads overlap the previous chunk's work
         auto tok_of = [&](int cc) { const int jj = cc * p.tpc + t; return jj < count ? toks[jj] : -1; };
         int tok_cur = tok_of(0), tok_nxt = nchunks > 1 ? tok_of(1) : -1;
-        float qn_cur = tok_cur >= 0 ? qn_row[tok_cur] : 0.f;
+        float sh_cur = tok_cur >= 0 ? shift_row[tok_cur] : 0.f;
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             const uint32_t use = (uint32_t)(c >> 1);
             const int tok_nn = c + 2 < nchunks ? tok_of(c + 2) : -1;
-            const float qn_nxt = tok_nxt >= 0 ? qn_row[tok_nxt] : 0.f;
+            const float sh_nxt = tok_nxt >= 0 ? shift_row[tok_nxt] : 0.f;
             const bool ok = mbar_wait(&s_full[buf], use & 1u, wc, code0 + 5);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const bool valid = tok_cur >= 0;
             const int i = valid ? tok_cur : 0;
             const int cmax = valid ? (((i >> 7) == n) ? (i & 127) : 127) : -1;
-            const float mh = valid ? p.bound * qn_cur * kmx : 0.f;
+            const float mh = valid ? sh_cur : 0.f;
             tok_cur = tok_nxt;
             tok_nxt = tok_nn;
-            qn_cur = qn_nxt;
+            sh_cur = sh_nxt;
             const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 128u);
             float l = 0.f;
 #pragma unroll
@@ -314,57 +323,21 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
 }
 
-// |q| per computed query row (rows q0 .. T-1); D/8 lanes per row (a
-// streaming read of Q).
-template <int D>
-__global__ void __launch_bounds__(256) fwd_qnorm_kernel(const __nv_bfloat16* __restrict__ q, int B, int T, int Hq,
-                                                        int q0, float* __restrict__ qn)
-{
-    constexpr int LPR = D / 8;
-    const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t ar = gt / LPR;
-    const int sub = (int)(gt % LPR);
-    const bool ok = ar < (int64_t)B * (T - q0) * Hq;
-    const int64_t row = ok ? active_row(ar, T, Hq, q0) : 0;
-    float ss = 0.f;
-    if (ok) {
-        const uint4 u = *reinterpret_cast<const uint4*>(q + row * D + sub * 8);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h2[e]);
-            ss = fmaf(f.x, f.x, ss);
-            ss = fmaf(f.y, f.y, ss);
-        }
-    }
-#pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if (ok && sub == 0) {
-        const int h = (int)(row % Hq);
-        const int64_t bi = row / Hq;
-        const int i = (int)(bi % T), b = (int)(bi / T);
-        qn[((int64_t)b * Hq + h) * T + i] = sqrtf(ss);
-    }
-}
-
-// max |k| per (b, group): grid (ceil(T / kKRows), B*Hkv); each CTA reduces its
-// rows to one value before a single atomic max (non-negative floats order like
-// their bits).
-constexpr int kKRows = 512;
-
+// max |k_j| per KV block: grid (nblk, B*Hkv), one CTA per block of 128 keys
+// (keys past T are not read); D/8 lanes per key row.
 template <int D>
 __global__ void __launch_bounds__(256) fwd_kmax_kernel(const __nv_bfloat16* __restrict__ k, int T, int Hkv,
-                                                       uint32_t* __restrict__ kmax_bits)
+                                                       int nblk, float* __restrict__ kmax_blk)
 {
     constexpr int LPR = D / 8, RPP = 256 / LPR;   // lanes per row, rows per pass
     __shared__ float red[8];
-    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
+    const int n = blockIdx.x, bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv;
     const int sub = threadIdx.x % LPR, r = threadIdx.x / LPR;
     float mx = 0.f;
     // the same number of passes for every lane: the shuffles below need the
     // whole warp, and rows past T are predicated off instead
-    for (int pass = 0; pass < kKRows / RPP; ++pass) {
-        const int t = blockIdx.x * kKRows + pass * RPP + r;
+    for (int pass = 0; pass < 128 / RPP; ++pass) {
+        const int t = n * 128 + pass * RPP + r;
         float ss = 0.f;
         if (t < T) {
             const uint4 u = *reinterpret_cast<const uint4*>(k + (((int64_t)b * T + t) * Hkv + g) * D + sub * 8);
@@ -387,23 +360,81 @@ __global__ void __launch_bounds__(256) fwd_kmax_kernel(const __nv_bfloat16* __re
     if (threadIdx.x == 0) {
         float m = red[0];
         for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
-        atomicMax(&kmax_bits[bg], __float_as_uint(sqrtf(m)));
+        kmax_blk[(int64_t)bg * nblk + n] = sqrtf(m);
     }
 }
 
-// O = O_acc / l (bf16), L = bound + log(l) for the computed rows (q0 ..
-// T-1); rows whose l underflowed are listed.
+// Per-row softmax shift m_i (log2 units) for the computed rows q0 .. T-1:
+// one warp per (b, group, query i) serves the G heads of the group, which
+// share the selection.  U = |c1| |q| max over the selected blocks of their
+// max |k|; S_ii = c1 q_i . k_i (the own key); m = min(U, S_ii + slack).
+// Selection entries outside [0, i/128] are skipped here (the inverse index
+// reports them).
+template <int D>
+__global__ void __launch_bounds__(256) fwd_shift_kernel(const __nv_bfloat16* __restrict__ q,
+                                                        const __nv_bfloat16* __restrict__ k,
+                                                        const int32_t* __restrict__ idx,
+                                                        const int32_t* __restrict__ nsel,
+                                                        const float* __restrict__ kmax_blk, int B, int T, int Hq,
+                                                        int Hkv, int topk, int nblk, int q0, float c1,
+                                                        float* __restrict__ shift)
+{
+    constexpr int EPL = D / 32;   // elements per lane
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int Tq = T - q0;
+    if (w >= (int64_t)B * Hkv * Tq) return;   // warp-uniform
+    const int bg = (int)(w / Tq), i = q0 + (int)(w % Tq);
+    const int b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+    const int64_t srow = (int64_t)bg * T + i;
+    int ns = nsel[srow];
+    ns = ns < 0 ? 0 : (ns > topk ? topk : ns);
+    float km = 0.f;
+    for (int s = lane; s < ns; s += 32) {
+        const int n = idx[srow * topk + s];
+        if (n >= 0 && n <= (i >> 7)) km = fmaxf(km, kmax_blk[(int64_t)bg * nblk + n]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, off));
+    float kv[EPL];
+    {
+        const __nv_bfloat16* kr = k + (((int64_t)b * T + i) * Hkv + g) * D + lane * EPL;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) kv[e] = __bfloat162float(kr[e]);
+    }
+    const float c1abs = fabsf(c1);
+    for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        const __nv_bfloat16* qr = q + (((int64_t)b * T + i) * Hq + h) * D + lane * EPL;
+        float ss = 0.f, dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            const float x = __bfloat162float(qr[e]);
+            ss = fmaf(x, x, ss);
+            dot = fmaf(x, kv[e], dot);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        }
+        if (lane == 0)
+            shift[((int64_t)b * Hq + h) * T + i] = fminf(c1abs * sqrtf(ss) * km, c1 * dot + kShiftSlack);
+    }
+}
+
+// O = O_acc / l (bf16), L = (m + log2 l) ln 2 for the computed rows (q0 ..
+// T-1); rows whose l is outside [kSumLow, kSumHigh] or not finite are listed
+// (count in status word 2).
 template <int D>
 __global__ void __launch_bounds__(256) fwd_finalize_kernel(const float* __restrict__ oacc,
                                                            const float* __restrict__ lacc,
-                                                           const float* __restrict__ qn,
-                                                           const float* __restrict__ kmax, int B, int T,
-                                                           int Hq, int Hkv, int q0, float abs_scale,
-                                                           __nv_bfloat16* __restrict__ o,
-                                                           float* __restrict__ lse, int* nflag,
-                                                           int* flags)
+                                                           const float* __restrict__ shift, int B, int T,
+                                                           int Hq, int q0, __nv_bfloat16* __restrict__ o,
+                                                           float* __restrict__ lse, uint32_t* nflag, int* flags)
 {
     constexpr int LPR = D / 8;
+    constexpr float kLn2 = 0.6931471805599453f;
     const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t ar = gt / LPR;
     const int sub = (int)(gt % LPR);
@@ -412,7 +443,6 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const float* __restri
     const int h = (int)(row % Hq);
     const int64_t bi = row / Hq;
     const int i = (int)(bi % T), b = (int)(bi / T);
-    const int G = Hq / Hkv;
     const int64_t lrow = ((int64_t)b * Hq + h) * T + i;
     const float l = lacc[lrow];
     const float inv = 1.f / l;
@@ -425,14 +455,13 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const float* __restri
     out.w = pack_bf16x2(c.z * inv, c.w * inv);
     *reinterpret_cast<uint4*>(o + row * D + sub * 8) = out;
     if (sub == 0) {
-        const float mh = abs_scale * qn[lrow] * kmax[b * Hkv + h / G];
-        lse[lrow] = mh + logf(l);
-        if (!(l >= kUnderflow)) flags[atomicAdd(nflag, 1)] = (int)row;
+        lse[lrow] = (shift[lrow] + log2f(l)) * kLn2;
+        if (!(l >= kSumLow && l <= kSumHigh)) flags[atomicAdd(nflag, 1u)] = (int)row;
     }
 }
 
-// Exact two-pass softmax for the listed rows (rare: bound far above the true
-// maximum).  One warp per row.
+// Exact two-pass softmax for the listed rows (rare: a row whose best score is
+// more than the shift slack above its own key's score).  One warp per row.
 template <int D>
 __global__ void __launch_bounds__(128) fwd_fallback_kernel(const __nv_bfloat16* __restrict__ q,
                                                            const __nv_bfloat16* __restrict__ k,
@@ -440,7 +469,7 @@ __global__ void __launch_bounds__(128) fwd_fallback_kernel(const __nv_bfloat16* 
                                                            const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ nsel, int B, int T,
                                                            int Hq, int Hkv, int topk, float scale,
-                                                           const int* nflag, const int* flags,
+                                                           const uint32_t* nflag, const int* flags,
                                                            __nv_bfloat16* __restrict__ o,
                                                            float* __restrict__ lse)
 {
@@ -448,7 +477,7 @@ __global__ void __launch_bounds__(128) fwd_fallback_kernel(const __nv_bfloat16* 
     __shared__ float ps[4][32];
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = Hq / Hkv;
-    const int nf = *nflag;
+    const int nf = (int)*nflag;
     for (int f = blockIdx.x * 4 + w; f < nf; f += gridDim.x * 4) {
         const int64_t row = flags[f];
         const int h = (int)(row % Hq);
@@ -519,38 +548,37 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
                          cudaStream_t st)
 {
     uint8_t* w = (uint8_t*)ws;
-    float* qn = (float*)(w + L.qnorm);
+    float* shift = (float*)(w + L.shift);
     float* kmax = (float*)(w + L.kmax);
     float* oacc = (float*)(w + L.oacc);
     float* lacc = (float*)(w + L.lacc);
-    int* nflag = (int*)(w + L.nflag);
+    uint32_t* nflag = (uint32_t*)(w + L.status) + 2;   // cleared with the status words by the caller
     int* flags = (int*)(w + L.flags);
     const __nv_bfloat16* qb = (const __nv_bfloat16*)q;
     const __nv_bfloat16* kb = (const __nv_bfloat16*)k;
+    const float c1 = pr.scale * kLog2e;
     cudaError_t e;
-    if ((e = cudaMemsetAsync(kmax, 0, sizeof(float) * pr.B * pr.Hkv, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(oacc, 0, sizeof(float) * (size_t)pr.rows_q() * D, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(lacc, 0, sizeof(float) * (size_t)pr.rows_q(), st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(nflag, 0, sizeof(int), st)) != cudaSuccess) return e;
 
-    const int64_t th = pr.rows_q_active() * (D / 8);
-    fwd_qnorm_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(qb, pr.B, pr.T, pr.Hq, pr.q0, qn);
+    fwd_kmax_kernel<D><<<dim3((unsigned)pr.nblk, (unsigned)(pr.B * pr.Hkv)), 256, 0, st>>>(kb, pr.T, pr.Hkv,
+                                                                                      pr.nblk, kmax);
     count_launches(1);
-    dim3 gk((unsigned)((pr.T + kKRows - 1) / kKRows), (unsigned)(pr.B * pr.Hkv));
-    fwd_kmax_kernel<D><<<gk, 256, 0, st>>>(kb, pr.T, pr.Hkv, (uint32_t*)kmax);
+    const int64_t warps = (int64_t)pr.B * pr.Hkv * (pr.T - pr.q0);
+    fwd_shift_kernel<D><<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(qb, kb, idx, nsel, kmax, pr.B, pr.T, pr.Hq,
+                                                                    pr.Hkv, pr.topk, pr.nblk, pr.q0, c1, shift);
     count_launches(1);
 
     FwdParams p;
     p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
     p.lgG = 31 - __builtin_clz((unsigned)pr.G);
     p.tpc = 128 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;
-    p.c1 = pr.scale * kLog2e;
-    p.bound = fabsf(pr.scale) * kLog2e;
+    p.c1 = c1;
     p.q = qb;
     p.ptr = (const int32_t*)(w + L.ptr);
     p.off = (const int32_t*)(w + L.cnt);
     p.tok = (const int32_t*)(w + L.tok);
-    p.qn = qn; p.kmax = kmax; p.oacc = oacc; p.lacc = lacc;
+    p.shift = shift; p.oacc = oacc; p.lacc = lacc;
     p.status = (uint32_t*)(w + L.status);
     p.RB = range_blocks(pr);
     p.qb0 = pr.qb0;
@@ -566,8 +594,7 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
 
     const int64_t fth = pr.rows_q_active() * (D / 8);
     fwd_finalize_kernel<D><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(
-        oacc, lacc, qn, kmax, pr.B, pr.T, pr.Hq, pr.Hkv, pr.q0, fabsf(pr.scale), (__nv_bfloat16*)o, lse, nflag,
-        flags);
+        oacc, lacc, shift, pr.B, pr.T, pr.Hq, pr.q0, (__nv_bfloat16*)o, lse, nflag, flags);
     count_launches(1);
     fwd_fallback_kernel<D><<<148, 128, 0, st>>>(qb, kb, (const __nv_bfloat16*)v, idx, nsel, pr.B,
                                                 pr.T, pr.Hq, pr.Hkv, pr.topk, pr.scale, nflag, flags,

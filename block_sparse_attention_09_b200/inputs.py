@@ -16,6 +16,9 @@ one stream per tensor, then rounded to bf16):
   overwritten by ``alpha (cos w_f t, sin w_f t)``, f = 0..3,
   ``w_f = 2 pi / (4096 * 4**f)``, alpha = 2, so the proxy score of (i, j)
   gains ``alpha**2 sum_f cos(w_f (i - j))``, which favours nearby blocks.
+* ``k_outliers=N`` (large-norm key variant): in every (batch, group), N key
+  rows at seeded positions are multiplied by 8 (about 8x the norm of the
+  others, as attention-sink-like keys of trained models have).
 * ``exact_proxy=True``: proxy values are put on the grid k/8 (|k| <= 64) after
   the recipe.  Every product is then a multiple of 1/64 and every partial sum
   of <= 64 products fits a float32 mantissa, so the proxy scores are exact in
@@ -42,6 +45,7 @@ class Config:
     dp: int
     topk: int
     bias: str = "none"   # "none" | "group" | "recency"
+    k_outliers: int = 0  # large-norm (x8) key rows per (batch, group)
 
     @property
     def Hp(self) -> int:
@@ -69,7 +73,7 @@ CONFIGS = {
 }
 
 # stream ids: one independent generator per tensor
-_STREAM = {"q": 1, "k": 2, "v": 3, "dout": 4, "qp": 5, "kp": 6, "bias_u": 7, "bias_c": 8}
+_STREAM = {"q": 1, "k": 2, "v": 3, "dout": 4, "qp": 5, "kp": 6, "bias_u": 7, "bias_c": 8, "outlier": 9}
 
 
 def _gen(seed: int, name: str) -> torch.Generator:
@@ -118,7 +122,14 @@ def make_inputs(cfg: Config, seed: int = 0, exact_proxy: bool = False, parts=Non
     for name, H, D in (("q", cfg.Hq, cfg.d), ("k", cfg.Hkv, cfg.d), ("v", cfg.Hkv, cfg.d),
                        ("dout", cfg.Hq, cfg.d)):
         if name in want:
-            out[name] = _randn((B, T, H, D), seed, name).to(torch.bfloat16).contiguous()
+            x = _randn((B, T, H, D), seed, name)
+            if name == "k" and cfg.k_outliers > 0:
+                g = _gen(seed, "outlier")
+                for b in range(B):
+                    for h in range(H):
+                        pos = torch.randperm(T, generator=g)[:cfg.k_outliers]
+                        x[b, pos, h] *= 8.0
+            out[name] = x.to(torch.bfloat16).contiguous()
     if "qp" in want or "kp" in want:
         qp = _randn((B, T, cfg.Hp, cfg.dp), seed, "qp")
         kp = _randn((B, T, cfg.Hp, cfg.dp), seed, "kp")

@@ -70,6 +70,8 @@ def _load():
     lib.msa_decode.restype = I
     lib.msa_f32_to_bf16.argtypes = [P, P, ctypes.c_int64, P]
     lib.msa_f32_to_bf16.restype = I
+    lib.msa_fallback_rows.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.msa_fallback_rows.restype = I
     lib.msa_kernel_launches.argtypes = []
     lib.msa_kernel_launches.restype = U64
     for f in ("msa_proxy_select", "msa_fwd", "msa_bwd", "msa_check_status", "msa_diag_umma",
@@ -119,6 +121,14 @@ def check_status(ws: torch.Tensor, stream=None) -> int:
     code = ctypes.c_uint32(0)
     rc = LIB.msa_check_status(_p(ws), _stream(stream), ctypes.byref(code))
     return rc
+
+
+def fallback_rows(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise and read how many rows the last forward on ``ws`` redid
+    with its exact two-pass softmax."""
+    n = ctypes.c_int64(0)
+    _check(LIB.msa_fallback_rows(_p(ws), _stream(stream), ctypes.byref(n)), "msa_fallback_rows")
+    return int(n.value)
 
 
 def _bf16(*ts):

@@ -230,6 +230,14 @@ MSA_API int msa_f32_to_bf16(const float* src, void* dst, int64_t n, void* stream
  * receives the raw device code (which wait or check failed). */
 MSA_API int msa_check_status(const void* ws, void* stream, uint32_t* code);
 
+/* Synchronises `stream`, then reads how many query rows the last msa_fwd /
+ * msa_fwd_ex on this workspace recomputed with its exact two-pass softmax
+ * (rows whose fixed softmax shift left their weights outside the fp32 range
+ * the forward accepts: only a row whose best score lies more than about
+ * 140 nats above the score of the query's own key).
+ * Any later call on the same workspace resets the count. */
+MSA_API int msa_fallback_rows(const void* ws, void* stream, int64_t* rows);
+
 /* Human-readable text for a status code (static storage). */
 MSA_API const char* msa_strerror(int status);
 
@@ -254,9 +262,8 @@ MSA_API uint64_t msa_kernel_launches(void);
  * operands staged the way the kernels stage them.  A: [128][K] bf16, B:
  * [N][K] bf16, D: [128][N] fp32, all device pointers.  mode: 0 = A,B K-major
  * in shared memory; 1 = A K-major, B MN-major; 2 = A,B MN-major; 3 = A in
- * tensor memory, B MN-major; 4 = A in tensor memory, B K-major; adding 8
- * exchanges the two byte offsets of the MN-major descriptors (a check that
- * the convention in use is the right one).  N in {64,128}, K in {64,128};
+ * tensor memory, B MN-major; 4 = A in tensor memory, B K-major.
+ * N in {64,128}, K in {64,128};
  * `ws` needs 256 bytes.  Synchronous. */
 MSA_API int msa_diag_umma(int mode, int N, int K, const void* A, const void* B, float* D, void* ws,
                   void* stream);

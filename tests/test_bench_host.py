@@ -2,6 +2,7 @@
 the (query head, key) pairs the oracle's own selection reads, and the guard
 that reports recorded DRAM traffic only for unchanged kernel sources."""
 import hashlib
+import json
 import os
 import sys
 
@@ -61,13 +62,17 @@ def test_recorded_traffic_needs_unchanged_sources(tmp_path, monkeypatch):
     (csrc / "a.cu").write_bytes(b"kernel source")
     (csrc / "b.h").write_bytes(b"header")
     digest = hashlib.sha256(b"kernel source" + b"header").hexdigest()
-    (tmp_path / "profiles" / "dram_msa_w.md").write_text(
-        f"text\n```\ntraffic k1 123456 a.cu,b.h {digest}\ntraffic k2 5 a.cu 00\n```\n")
+    rec = {"records": [
+        {"kernel": "k1", "workload": "w", "bytes_per_launch_captured": 15432.0, "scale_to_full": 8.0,
+         "sources": ["a.cu", "b.h"], "sources_sha256": digest},
+        {"kernel": "k2", "workload": "w", "bytes_per_launch_captured": 5.0, "scale_to_full": 1.0,
+         "sources": ["a.cu"], "sources_sha256": "00"}]}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.recorded_traffic("k1", "w") == 123456.0
     assert bench.recorded_traffic("k2", "w") is None          # hash differs
     assert bench.recorded_traffic("k3", "w") is None          # no record
-    assert bench.recorded_traffic("k1", "other") is None      # no summary for the workload
+    assert bench.recorded_traffic("k1", "other") is None      # no record for the workload
     (csrc / "a.cu").write_bytes(b"kernel source, edited")
     assert bench.recorded_traffic("k1", "w") is None          # changed since the capture
 

@@ -6,7 +6,7 @@ dK/dV -- against the oracle run on the unsplit sequence.
 
 The per-rank attention here is the oracle behind the library's call
 signatures (a test stand-in: on GPUs the same orchestration calls the CUDA
-library, checked in test_gpu_cp.py); what these tests pin is the
+library, checked in test_gpu_zz_cp.py); what these tests pin is the
 decomposition and the collectives, with a real process group.
 """
 import os

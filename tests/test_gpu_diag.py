@@ -23,18 +23,6 @@ def test_umma_staging_matches_matmul(msa, mode, N, K):
     assert err <= 1e-3 * ref.abs().max().item() + 1e-3, (mode, N, K, err)
 
 
-@pytest.mark.parametrize("mode", [1, 2, 3])
-def test_exchanged_mn_offsets_are_wrong(msa, mode):
-    """The other assignment of the two MN-major byte offsets must NOT
-    reproduce the product (so the convention in use is the checked one)."""
-    g = torch.Generator().manual_seed(7 + mode)
-    A = torch.randn(128, 128, generator=g).to(torch.bfloat16)
-    B = torch.randn(128, 128, generator=g).to(torch.bfloat16)
-    ref = A.float() @ B.float().T
-    D = msa.diag_umma(mode + 8, A.cuda(), B.cuda()).cpu()
-    assert (D - ref).abs().max().item() > 1.0
-
-
 def test_bounded_wait_gives_up(msa):
     # a barrier nothing arrives on: the wait must end by itself with a timeout status
     rc = msa.diag_wait_timeout(20_000_000)

@@ -10,6 +10,17 @@ query rows, dK and dV of the last KV blocks (whose selecting queries the
 oracle can enumerate) -- and, over the whole tensors, identities that hold at
 any size: softmax rows sum to one, so sum_j dV_j = sum_{i,h} dO_ih per group,
 and sum_j dS_ij = 0, so sum_j dK_j = 0.
+
+A second backward, in the same launch configuration, takes dO restricted to
+a seeded set S of query tokens spread over the whole sequence (dO = 0
+elsewhere).  Rows outside S then contribute exactly zero to every gradient
+(dV gains P * 0, and dS = P (dO.v - dO.O) = 0), so dK and dV of ANY block are
+sums over the S rows that selected it, which the oracle enumerates from its
+own selection of those rows.  That checks, element by element and with the
+unrounded fp32 dK/dV (MSA_DKV_F32) against the plain max-abs bound 2e-2, the
+heavily shared blocks -- block 0, the block the S rows select most, a
+mid-sequence block -- whose partials arrive from every query range of the
+kernels' work items; dQ of every row outside S must be exactly zero.
 """
 import numpy as np
 import pytest
@@ -22,8 +33,8 @@ from parity_util import compare, f32, odims, to_dev
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
-@pytest.mark.parametrize("name,nsel_rows,nq_rows", [("32k", 256, 512), ("128k", 192, 384)])
-def test_full_size(name, nsel_rows, nq_rows):
+@pytest.mark.parametrize("name,nsel_rows,nq_rows,s_tokens", [("32k", 256, 512, 1024), ("128k", 192, 384, 512)])
+def test_full_size(name, nsel_rows, nq_rows, s_tokens):
     from block_sparse_attention_09_b200 import msa
     cfg = CONFIGS[name]
     inp = make_inputs(cfg, seed=11, exact_proxy=True)
@@ -62,7 +73,7 @@ def test_full_size(name, nsel_rows, nq_rows):
     r = np.array(qrows)
     h, b, i = (r // T) % Hq, r // (T * Hq), r % T
     compare("O rows", f32(o)[b, i, h], oo[b, i, h])
-    compare("L rows", f32(lse)[b, h, i], lo[b, h, i])
+    compare("L rows", f32(lse)[b, h, i], lo[b, h, i], rel=0.0)
     compare("dQ rows", f32(dq)[b, i, h], dqo[b, i, h])
 
     # ---- dK, dV of the last two KV blocks of every group: their selecting
@@ -93,3 +104,54 @@ def test_full_size(name, nsel_rows, nq_rows):
             assert np.abs(kk.sum(0)).max() <= tol_k, ("sum dK", np.abs(kk.sum(0)).max(), tol_k)
             want = dout[bb][:, g * G:(g + 1) * G].sum((0, 1))
             assert np.abs(vv.sum(0) - want).max() <= tol_v, ("sum dV", np.abs(vv.sum(0) - want).max(), tol_v)
+
+    # ---- masked dO: heavily shared blocks, fp32 dK/dV, strict bound
+    masked_dkdv_check(cfg, inp, x, dev, idx, nsel, o, lse, ws, s_tokens)
+
+
+def masked_dkdv_check(cfg, inp, x, dev, idx, nsel, o, lse, ws, s_tokens):
+    from block_sparse_attention_09_b200 import msa
+    m = odims(cfg)
+    T, G, Hq, Hkv, nb = cfg.T, cfg.G, cfg.Hq, cfg.Hkv, m.nblk
+    toks = np.array(sample_rows(T, s_tokens, seed=21, must=[0, T // 2, T - 1]), dtype=np.int64)
+    keep = np.zeros(T, dtype=np.float32)
+    keep[toks] = 1.0
+    dout_m = inp["dout"].float() * torch.from_numpy(keep).view(1, T, 1, 1)
+    dout_m = dout_m.to(torch.bfloat16)
+    dq_m, dk_m, dv_m = msa.bwd(dev["q"], dev["k"], dev["v"], o, dout_m.cuda(), lse, idx, nsel, ws=ws, check=True,
+                               reuse_index=True, dkv_f32=True)
+    torch.cuda.synchronize()
+    assert dk_m.dtype == torch.float32
+    # rows outside S: dQ exactly zero
+    outside = np.ones(T, dtype=bool)
+    outside[toks] = False
+    assert not f32(dq_m)[:, outside].any(), "dQ of rows with dO = 0 is not zero"
+
+    # the oracle on the S rows only: its own selection, O, L, D
+    srows = [(b * Hkv + g) * T + int(t) for b in range(cfg.B) for g in range(Hkv) for t in toks]
+    idx_s, nsel_s, _ = O.select(m, x["qp"], x["kp"], rows=srows)
+    qrows = [(b * Hq + g * G + hh) * T + int(t) for b in range(cfg.B) for g in range(Hkv) for hh in range(G)
+             for t in toks]
+    xm = dict(x)
+    xm["dout"] = dout_m.float().numpy()
+    o_s, l_s = O.fwd(m, x["q"], x["k"], x["v"], idx_s, nsel_s, rows=qrows)
+    _, D_s = O.bwd_dq(m, x["q"], x["k"], x["v"], xm["dout"], o_s, l_s, idx_s, nsel_s, rows=qrows)
+    blocks, spans = [], []
+    for b in range(cfg.B):
+        for g in range(Hkv):
+            sel = idx_s[b, g, toks]                           # [S, topk]
+            counts = np.bincount(sel[sel >= 0].ravel(), minlength=nb)
+            for n in sorted({0, int(counts.argmax()), nb // 2}):
+                who = toks[(sel == n).any(axis=1)]
+                # the query eighths of the sequence its S partials come from
+                spans.append(len(set((who * 8 // T).tolist())))
+                blocks.append((b * Hkv + g) * nb + n)
+    assert max(spans) >= 4, ("shared blocks receive partials from few query ranges", spans)
+    dko, dvo = O.bwd_dkdv(m, x["q"], x["k"], x["v"], xm["dout"], l_s, D_s, idx_s, nsel_s, blocks=blocks)
+    gk, gv = f32(dk_m), f32(dv_m)
+    for bl in blocks:
+        n = bl % nb
+        b, g = divmod(bl // nb, Hkv)
+        sl = slice(n * 128, min((n + 1) * 128, T))
+        compare(f"dK32 blk {n} g{g}", gk[b, sl, g], dko[b, sl, g], rel=0.0)
+        compare(f"dV32 blk {n} g{g}", gv[b, sl, g], dvo[b, sl, g], rel=0.0)
