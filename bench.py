@@ -346,10 +346,10 @@ def run_decode(args, cfg, rank, local):
 
 
 def run_cp(args, cfg, rank, local, world):
-    """Context-parallel step: the workload's sequence split into equal 128-row
-    shards over the ranks (block_sparse_attention_09_b200.cp): all-gather of
-    k, v, kp, each rank's selection, forward and backward of its own query
-    rows, reduce-scatter of the fp32 partial dK/dV.  The work is fixed as the
+    """Context-parallel step: the workload's sequence split into zig-zag
+    chunks of 128-row blocks over the ranks (block_sparse_attention_09_b200.cp):
+    all-gather of k, v, kp, each rank's selection, forward and backward of its
+    own query rows, reduce-scatter of the fp32 partial dK/dV.  The work is fixed as the
     ranks grow (strong scaling); value = FLOPs of the whole sequence's step /
     the slowest rank's time."""
     import torch
@@ -361,9 +361,9 @@ def run_cp(args, cfg, rank, local, world):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
-    r0, r1 = cp.shard_bounds(cfg.T, world, rank)
+    chunks = cp.shard_chunks(cfg.T, world, rank)
     host = make_inputs(cfg, seed=0)   # the same sequence on every rank; each keeps its rows
-    d = {k: v[:, r0:r1].contiguous().to(dev) for k, v in host.items()}
+    d = {k: cp.take_rows(v, chunks).to(dev) for k, v in host.items()}
     del host
 
     def step():
@@ -371,8 +371,12 @@ def run_cp(args, cfg, rank, local, world):
 
     out = step()
     nsel = out[6]
-    # selected-key pairs of this rank's rows, summed over the ranks
-    pairs = torch.tensor([pair_count(cfg, nsel, r0)["pairs"]], dtype=torch.float64, device=dev)
+    # selected-key pairs of this rank's rows (chunk by chunk), summed over the ranks
+    own, at = 0.0, 0
+    for c0, c1 in chunks:
+        own += pair_count(cfg, nsel[:, :, at:at + c1 - c0], c0)["pairs"]
+        at += c1 - c0
+    pairs = torch.tensor([own], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(pairs)
     f_proxy, f_fwd, f_bwd = flops_from_nsel(cfg, {"pairs": float(pairs.item())})
@@ -408,7 +412,7 @@ def run_cp(args, cfg, rank, local, world):
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded N(0,1) bf16 inputs" + (", planted local-recency proxy bias" if cfg.bias == "recency" else ""),
-            "config": {"workload": workload_name(cfg) + f", rows split over {world} ranks",
+            "config": {"workload": workload_name(cfg) + f", rows split over {world} ranks (zig-zag chunks)",
                        "B": cfg.B, "T": cfg.T, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "dp": cfg.dp,
                        "topk": cfg.topk, "parallelism": f"cp{world}",
                        "l2": "inputs larger than L2, no flush"},

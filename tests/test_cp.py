@@ -83,17 +83,37 @@ class OracleOps:
         return x.to(torch.bfloat16)
 
 
-def test_shard_bounds_cover_the_sequence():
-    for T in (1, 127, 128, 640, 1000, 4096, 131072 + 77):
+def test_shard_chunks_cover_the_sequence_and_balance_the_work():
+    for T in (1, 127, 128, 640, 1000, 4096, 131072 + 77, 1 << 20):
         for world in (1, 2, 3, 4, 8):
-            b = [cp.shard_bounds(T, world, r) for r in range(world)]
-            assert b[0][0] == 0 and b[-1][1] == T
-            for (a0, a1), (c0, c1) in zip(b, b[1:]):
-                assert a1 == c0                      # contiguous
-            for r0, r1 in b:
-                assert r0 % 128 == 0 and r0 <= r1    # block aligned
-            nb = [(r1 - r0 + 127) // 128 for r0, r1 in b]
-            assert max(nb) - min(nb) <= 1            # balanced by whole blocks
+            chunks = [cp.shard_chunks(T, world, r) for r in range(world)]
+            flat = sorted(c for ch in chunks for c in ch)
+            assert flat[0][0] == 0 and flat[-1][1] == T
+            for (a0, a1), (c0, c1) in zip(flat, flat[1:]):
+                assert a1 == c0                       # contiguous, disjoint
+            for c0, c1 in flat:
+                assert c0 % 128 == 0 and c0 < c1      # block aligned, non-empty
+            for ch in chunks:
+                assert ch == sorted(ch)               # a rank's rows in sequence order
+            nblk = (T + 127) // 128
+            if nblk >= 2 * world:
+                # rows: within two blocks of each other
+                nb = [sum((c1 - c0 + 127) // 128 for c0, c1 in ch) for ch in chunks]
+                assert max(nb) - min(nb) <= 2
+                # causal proxy work (keys scored per row ~ its position): the
+                # zig-zag pairing keeps every rank within 2 % + two chunks'
+                # rounding of the mean
+                work = [sum(i for c0, c1 in ch for i in range(c0, c1, 128)) for ch in chunks]
+                mean = sum(work) / world
+                assert max(work) <= mean * 1.02 + 2 * 128 * nblk, (T, world, work)
+
+
+def test_zigzag_pairs_early_and_late_chunks():
+    ch = [cp.shard_chunks(16 * 128, 4, r) for r in range(4)]
+    assert ch[0] == [(0, 256), (1792, 2048)]
+    assert ch[3] == [(768, 1024), (1024, 1280)]
+    x = torch.arange(16 * 128).view(1, -1)
+    assert cp.take_rows(x, ch[1]).tolist()[0] == list(range(256, 512)) + list(range(1536, 1792))
 
 
 CFG = Config("cp", B=1, T=1000, Hq=4, Hkv=2, d=64, dp=32, topk=3)
@@ -112,11 +132,11 @@ def _rank_main(rank, world, port, out_dir):
                             timeout=timedelta(seconds=120))
     try:
         x = make_inputs(CFG, seed=3, exact_proxy=True)
-        r0, r1 = cp.shard_bounds(CFG.T, world, rank)
-        mine = {k: t[:, r0:r1].contiguous() for k, t in x.items()}
+        chunks = cp.shard_chunks(CFG.T, world, rank)
+        mine = {k: cp.take_rows(t, chunks) for k, t in x.items()}
         o, lse, dq, dk, dv = cp.step(mine["q"], mine["k"], mine["v"], mine["dout"], mine["qp"], mine["kp"],
                                      CFG.topk, CFG.T, ops=OracleOps)
-        torch.save(dict(r0=r0, r1=r1, o=o, lse=lse, dq=dq, dk=dk, dv=dv), os.path.join(out_dir, f"rank{rank}.pt"))
+        torch.save(dict(chunks=chunks, o=o, lse=lse, dq=dq, dk=dk, dv=dv), os.path.join(out_dir, f"rank{rank}.pt"))
     finally:
         dist.destroy_process_group()
 
@@ -148,16 +168,15 @@ def test_cp_step_matches_the_unsplit_sequence(tmp_path, oracle_mod, world):
     covered = 0
     for r in range(world):
         got = torch.load(tmp_path / f"rank{r}.pt")
-        r0, r1 = got["r0"], got["r1"]
-        covered += r1 - r0
-        sl = slice(r0, r1)
-        # bf16 outputs: within the rounding of one bf16 store (dK/dV: two
-        # shards' fp32 partials added before the one rounding)
-        for name, g, rf in (("o", got["o"], ref["o"][:, sl]), ("dq", got["dq"], ref["dq"][:, sl]),
-                            ("dk", got["dk"], ref["dk"][:, sl]), ("dv", got["dv"], ref["dv"][:, sl])):
+        rows = np.concatenate([np.arange(c0, c1) for c0, c1 in got["chunks"]])
+        covered += len(rows)
+        # bf16 outputs: within the rounding of one bf16 store (dK/dV: several
+        # chunks' fp32 partials added before the one rounding)
+        for name, g, rf in (("o", got["o"], ref["o"][:, rows]), ("dq", got["dq"], ref["dq"][:, rows]),
+                            ("dk", got["dk"], ref["dk"][:, rows]), ("dv", got["dv"], ref["dv"][:, rows])):
             err = np.abs(g.float().numpy() - rf)
             assert (err <= 1e-6 + 2.0 ** -8 * np.abs(rf)).all(), (name, r, float(err.max()))
-        assert np.allclose(got["lse"].numpy(), ref["lse"][:, :, sl], rtol=1e-6, atol=1e-5)
+        assert np.allclose(got["lse"].numpy(), ref["lse"][:, :, rows], rtol=1e-6, atol=1e-5)
     assert covered == CFG.T
 
 

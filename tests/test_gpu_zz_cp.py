@@ -1,8 +1,9 @@
 """GPU checks of the context-parallel pieces, on one GPU: the library calls
 restricted to a shard's query rows (q_begin) and the fp32 partial gradients,
-with the ranks of a context-parallel step run one after another (the
-all-gather is a slice of the whole tensors, the reduce-scatter a sum of the
-partials); the kernels of different ranks never wait on one another.
+with the ranks of a context-parallel step run one after another, one call
+per zig-zag chunk (the all-gather is a slice of the whole tensors, the
+reduce-scatter a sum of the partials); the kernels of different ranks never
+wait on one another.
 
 The sharded step must give the selection of the unsplit call bit for bit,
 O, L and dQ within two bf16 ulps of it (the fp32 reductions add in a
@@ -40,11 +41,12 @@ def test_sharded_step_matches_unsplit(name, cfg, world):
     idx, nsel = msa.proxy_select(x["qp"], x["kp"], cfg.topk, check=True)
     o, lse = msa.fwd(x["q"], x["k"], x["v"], idx, nsel, check=True)
     dq, dk, dv = msa.bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, idx, nsel, check=True)
-    # the ranks of a context-parallel step, one after another
-    bounds = [cp.shard_bounds(cfg.T, world, r) for r in range(world)]
+    # the ranks of a context-parallel step, one after another, each over its
+    # zig-zag chunks (one library call per chunk)
+    chunks = [c for r in range(world) for c in cp.shard_chunks(cfg.T, world, r)]
     dk_sum = torch.zeros(x["k"].shape, dtype=torch.float32, device="cuda")
     dv_sum = torch.zeros_like(dk_sum)
-    for r0, r1 in bounds:
+    for r0, r1 in chunks:
         mine = {k: t[:, r0:r1].contiguous() for k, t in x.items()}
         pre = {k: x[k][:, :r1].contiguous() for k in ("k", "v", "kp")}
         o_r, lse_r, dq_r, dk_p, dv_p, idx_r, nsel_r = cp.local_step(
