@@ -53,6 +53,8 @@ def parse():
                     help="override the workload's proxy-input structure (profiling variants)")
     ap.add_argument("--outliers", type=int, default=0,
                     help="large-norm (x8) key rows per (batch, group): the attention-sink-like variant")
+    ap.add_argument("--proxy-grad", action="store_true",
+                    help="also time the proxy-head gradient (forward keeping block masses + msa_proxy_bwd)")
     ap.add_argument("--groups", type=int, default=0,
                     help="run only this many of the workload's KV groups (same per-group shape; profiling "
                          "captures scale their counters by the group ratio)")
@@ -554,6 +556,44 @@ def main():
     phase_ms = {k: statistics.mean(v) for k, v in phase.items()}
     kern_ms = {kernel_names[k]: statistics.mean(a.elapsed_time(b_) for a, b_ in v) for k, v in kev.items()}
 
+    # ---- the proxy-head gradient (reported apart from the step's metric)
+    proxy_grad = None
+    if args.proxy_grad:
+        ws_pg = msa.proxy_workspace(dims, dev)
+        pg_out = (torch.empty(d["qp"].shape, dtype=torch.float32, device=dev),
+                  torch.empty(d["kp"].shape, dtype=torch.float32, device=dev),
+                  torch.empty((B, cfg.Hkv, T), dtype=torch.float32, device=dev))
+
+        def pg_step(ev=None):
+            ix, ns = msa.proxy_select(d["qp"], d["kp"], cfg.topk, ws=ws_sel)
+            if ev is not None:
+                ev[0].record(stream)
+            msa.fwd(d["q"], d["k"], d["v"], ix, ns, ws=ws_pg, out=(o, lse), block_mass=True)
+            if ev is not None:
+                ev[1].record(stream)
+            msa.bwd(d["q"], d["k"], d["v"], o, d["dout"], lse, ix, ns, ws=ws_pg, out=(dq, dk, dv), reuse_index=True)
+            if ev is not None:
+                ev[2].record(stream)
+            msa.proxy_bwd(d["q"], d["qp"], d["kp"], ix, ns, ws_pg, out=pg_out)
+            if ev is not None:
+                ev[3].record(stream)
+
+        pg_step()
+        if msa.check_status(ws_pg) != 0:
+            raise RuntimeError("device status after the proxy-head gradient")
+        for _ in range(args.warmup):
+            pg_step()
+        evs = []
+        for _ in range(args.steps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            evs.append(ev)
+            pg_step(ev)
+        torch.cuda.synchronize()
+        proxy_grad = {"fwd_with_block_mass_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+                      "proxy_bwd_ms": statistics.mean(e[2].elapsed_time(e[3]) for e in evs),
+                      "loss_sum": float(pg_out[2].double().sum().item())}
+        del ws_pg, pg_out
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -684,6 +724,7 @@ def main():
         "e2e": e2e,
         "gpu_launches": launches,
         "fallback_rows": fallback,
+        "proxy_grad": proxy_grad,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -15,6 +15,22 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 WsLayout ws_layout(const Problem& p, int which)
 {
+    if (which == MSA_PROXY_BWD) {
+        // the forward's layout (index, forward regions) at its own offsets,
+        // then the per-entry buffers of the proxy-head gradient past anything
+        // a forward or a main backward on the same workspace writes
+        WsLayout L = ws_layout(p, MSA_FWD);
+        const size_t bwd = ws_layout(p, MSA_BWD).total;
+        size_t off = L.total > bwd ? L.total : bwd;
+        auto take = [&](size_t bytes) { const size_t at = off; off = align256(off + bytes); return at; };
+        const size_t E = (size_t)p.B * p.Hp * p.T * p.topk;   // pair-list entries, at most
+        L.bmass = take(E * 2 * p.G * 4);
+        L.zsel = take(E * 2 * 4);
+        L.jsel = take(E * 2 * 4);
+        L.dz = take(E * 2 * 4);
+        L.total = off;
+        return L;
+    }
     WsLayout L;
     size_t off = 256;   // status words
     const size_t BH = (size_t)p.B * p.Hp;
@@ -25,6 +41,11 @@ WsLayout ws_layout(const Problem& p, int which)
         L.tot = take(BH * p.nblk * 4);
         L.ptr = take(BH * (p.nblk + 1) * 4);
         L.tok = take(BH * (size_t)p.T * p.topk * 4);
+        const size_t np = (size_t)pair_count(p.nblk);
+        L.cnt2 = take(BH * p.nblk * np * 4);
+        L.tot2 = take(BH * np * 4);
+        L.ptr2 = take(BH * (np + 1) * 4);
+        L.tok2 = take(BH * (size_t)p.T * p.topk * 4);
     }
     if (which == MSA_FWD) {
         L.shift = take(rows * 4);
@@ -159,7 +180,7 @@ size_t msa_workspace_size(const msa_dims* dims, int which)
 {
     Problem p;
     if (to_problem(dims, &p, which == MSA_DECODE) != MSA_OK) return 0;
-    if (which < MSA_SELECT || which > MSA_DECODE) return 0;
+    if (which < MSA_SELECT || which > MSA_PROXY_BWD) return 0;
     return ws_layout(p, which).total;
 }
 
@@ -196,7 +217,8 @@ int msa_fwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v
     int rc = to_problem(dims, &p);
     if (rc != MSA_OK) return rc;
     WsLayout L;
-    if ((rc = check_ws(p, MSA_FWD, ws, ws_bytes, &L)) != MSA_OK) return rc;
+    const bool mass = (flags & MSA_BLOCK_MASS) != 0;
+    if ((rc = check_ws(p, mass ? MSA_PROXY_BWD : MSA_FWD, ws, ws_bytes, &L)) != MSA_OK) return rc;
     if (empty(p)) return MSA_OK;
     if (!q || !k || !v || !idx || !nsel || !o || !lse) return MSA_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(idx, 16) || !aligned(nsel, 16) ||
@@ -212,7 +234,8 @@ int msa_fwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v
     if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     if (!(flags & MSA_REUSE_INDEX) && launch_block_index(p, idx, nsel, ws, L, st) != cudaSuccess)
         return MSA_ERR_LAUNCH;
-    if (launch_fwd(p, q, k, v, tk, tv, idx, nsel, o, lse, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    float* bmass = mass ? (float*)((uint8_t*)ws + L.bmass) : nullptr;
+    if (launch_fwd(p, q, k, v, tk, tv, idx, nsel, o, lse, ws, L, bmass, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     return MSA_OK;
 }
 
@@ -288,6 +311,29 @@ int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q, const v
     uint32_t* status = (uint32_t*)((uint8_t*)ws + L.status);
     if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     if (launch_decode(p, lens, q, qp, k, v, kp, idx, nsel, o, lse, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    return MSA_OK;
+}
+
+int msa_proxy_bwd(const msa_dims* dims, const void* qp, const void* kp, const int32_t* idx, const int32_t* nsel,
+                  float* dqp, float* dkp, float* loss, void* ws, size_t ws_bytes, void* stream)
+{
+    Problem p;
+    int rc = to_problem(dims, &p);
+    if (rc != MSA_OK) return rc;
+    WsLayout L;
+    if ((rc = check_ws(p, MSA_PROXY_BWD, ws, ws_bytes, &L)) != MSA_OK) return rc;
+    if (empty(p)) return MSA_OK;
+    if (!qp || !kp || !idx || !nsel || !dqp || !dkp || !loss) return MSA_ERR_NULL_PTR;
+    if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(idx, 16) || !aligned(nsel, 16) || !aligned(dqp, 16) ||
+        !aligned(dkp, 16) || !aligned(loss, 16))
+        return MSA_ERR_MISALIGNED;
+    if ((rc = check_device()) != MSA_OK) return rc;
+    CUtensorMap tk;
+    if (!make_tmap_bf16_4d(&tk, kp, p.dp, p.Hp, p.T, p.B, 64, 256)) return MSA_ERR_DRIVER;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t* status = (uint32_t*)((uint8_t*)ws + L.status);
+    if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return MSA_ERR_LAUNCH;
+    if (launch_proxy_bwd(p, tk, qp, kp, idx, nsel, dqp, dkp, loss, ws, L, st) != cudaSuccess) return MSA_ERR_LAUNCH;
     return MSA_OK;
 }
 

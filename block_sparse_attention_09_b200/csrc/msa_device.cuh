@@ -329,6 +329,72 @@ MSA_DEV RangeItem range_item(int x, int nblk, int RB, int qb0, int per_group, co
     return it;
 }
 
+// The forward walks the same ranges over PAIRS of KV blocks (2p, 2p+1): range
+// R holds the pairs p with 2p < qe.  The token segment comes from the pair
+// index (ptr2 [bg][npair+1], off2 [bg][qb][npair], valid for qb >= 2p); it.n
+// is the pair p.
+__host__ __device__ inline int pair_items_per_group(int nblk, int RB, int qb0)
+{
+    int total = 0;
+    for (int R = 0; qb0 + R * RB < nblk; ++R) total += (min(nblk, qb0 + (R + 1) * RB) + 1) / 2;
+    return total;
+}
+
+MSA_DEV RangeItem pair_item(int x, int nblk, int npair, int RB, int qb0, int per_group, const int32_t* ptr2,
+                            const int32_t* off2, int* qe_out)
+{
+    RangeItem it;
+    it.bg = x / per_group;
+    int rem = x % per_group, R = 0;
+    for (;;) {
+        const int np = (min(nblk, qb0 + (R + 1) * RB) + 1) / 2;
+        if (rem < np) break;
+        rem -= np;
+        ++R;
+    }
+    const int pn = rem, qs = qb0 + R * RB, qe = min(nblk, qb0 + (R + 1) * RB);
+    const int32_t* pp = ptr2 + (int64_t)it.bg * (npair + 1);
+    const int32_t* o = off2 + (int64_t)it.bg * nblk * npair;
+    const int base = pp[pn];
+    const int start = qs > 2 * pn ? o[(int64_t)qs * npair + pn] : 0;
+    const int end = qe >= nblk ? pp[pn + 1] - base : o[(int64_t)qe * npair + pn];
+    it.n = pn;
+    it.beg = base + start;
+    it.count = end - start;
+    *qe_out = qe;
+    return it;
+}
+
+// Block-membership masks of one query tile in shared memory: bit t of
+// mask[n*4 + t/32] says query qb*128 + t selected block n (n <= qb).  The
+// whole CTA calls it; returns false on a malformed row (entries outside
+// [0, i/128], not ascending, nsel outside [1, topk]), whose bad entries are
+// skipped.
+__device__ __forceinline__ bool build_masks(uint32_t* mask, const int32_t* idx, const int32_t* nsel, int T, int topk,
+                            int qb, int bg)
+{
+    const int nb = qb + 1;
+    for (int x = threadIdx.x; x < nb * 4; x += blockDim.x) mask[x] = 0u;
+    __syncthreads();
+    bool bad = false;
+    const int t = threadIdx.x, i = qb * 128 + t;
+    if (t < 128 && i < T) {
+        const int64_t row = (int64_t)bg * T + i;
+        int ns = nsel[row];
+        if (ns < 1 || ns > topk) { bad = true; ns = ns < 0 ? 0 : (ns > topk ? topk : ns); }
+        const int32_t* sel = idx + row * topk;
+        int prev = -1;
+        for (int s = 0; s < ns; ++s) {
+            const int n = sel[s];
+            if (n < 0 || n > qb || n <= prev) { bad = true; continue; }
+            prev = n;
+            atomicOr(&mask[n * 4 + (t >> 5)], 1u << (t & 31));
+        }
+    }
+    __syncthreads();
+    return !bad;
+}
+
 // Active query row r (0 .. B*(T-q0)*Hq - 1: the rows q0 .. T-1 of every batch
 // and head) -> its flat index (b*T + i)*Hq + h in a [B][T][Hq] tensor.
 MSA_DEV int64_t active_row(int64_t r, int T, int Hq, int q0)

@@ -34,10 +34,12 @@ struct Problem {
 // Byte offsets of the workspace regions.
 struct WsLayout {
     size_t status = 0;   // 256 B: [0] timeout code, [1] index error, [2] forward fallback rows
-    size_t cnt = 0, tot = 0, ptr = 0, tok = 0;   // block -> query inverse index
+    size_t cnt = 0, tot = 0, ptr = 0, tok = 0;       // block -> query inverse index
+    size_t cnt2 = 0, tot2 = 0, ptr2 = 0, tok2 = 0;   // block pair -> query (forward)
     size_t shift = 0, kmax = 0, oacc = 0, lacc = 0, flags = 0;   // forward
     size_t dsum = 0, dqacc = 0, dkacc = 0, dvacc = 0;   // backward
     size_t pooled = 0, part = 0;                        // decode
+    size_t bmass = 0, zsel = 0, jsel = 0, dz = 0;       // proxy-head gradient (per pair-list entry)
     size_t total = 0;
 };
 WsLayout ws_layout(const Problem& p, int which);
@@ -46,6 +48,9 @@ WsLayout ws_layout(const Problem& p, int which);
 // box and 128-byte swizzle.  Returns false if the driver refused it.
 bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t e0, uint64_t e1, uint64_t e2,
                        uint64_t e3, uint32_t box0, uint32_t box2);
+
+// Pairs of KV blocks (2p, 2p+1) of a sequence of nblk blocks.
+inline int pair_count(int nblk) { return (nblk + 1) / 2; }
 
 // Query blocks per work-item range of the Main Branch kernels.  The query-side
 // rows one range touches (fp32 accumulators and gathered bf16 inputs of a
@@ -99,10 +104,16 @@ cudaError_t launch_proxy_select(const Problem& p, const CUtensorMap& tm_qp, cons
 cudaError_t launch_block_index(const Problem& p, const int32_t* idx, const int32_t* nsel, void* ws,
                                const WsLayout& L, cudaStream_t st);
 
+// bmass (nullable): per pair-list entry, each selected block's weight sum per head
 cudaError_t launch_fwd(const Problem& p, const void* q, const void* k, const void* v,
                        const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int32_t* idx,
                        const int32_t* nsel, void* o, float* lse, void* ws, const WsLayout& L,
-                       cudaStream_t st);
+                       float* bmass, cudaStream_t st);
+
+// Proxy-head gradient from the pair index and block masses a forward left in ws.
+cudaError_t launch_proxy_bwd(const Problem& p, const CUtensorMap& tm_kp, const void* qp, const void* kp,
+                             const int32_t* idx, const int32_t* nsel, float* dqp, float* dkp, float* loss,
+                             void* ws, const WsLayout& L, cudaStream_t st);
 
 // dkv_f32: dk, dv are fp32 and receive the unrounded sums
 cudaError_t launch_bwd(const Problem& p, const void* q, const void* dout, const CUtensorMap& tm_k,

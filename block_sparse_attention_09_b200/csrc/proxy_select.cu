@@ -22,7 +22,9 @@
 // Selection state per row (shared memory, [slot][row] so a warp touches 32
 // distinct banks): a 4-ary heap of the best topk-1 (score, id) pairs whose
 // root is the worst kept pair, and a small pending list.  At the end each
-// warp sorts its rows' kept ids with a bitonic network across its lanes.  Key tiles are
+// selection thread sorts its own row's kept ids with a bitonic network in
+// registers (topk <= 64; larger topk: one row at a time across the warp's
+// lanes).  Key tiles are
 // scanned nearest-first (descending block id): under causal locality the
 // best blocks tend to be the recent ones, so after the first few tiles a
 // new tile rarely beats the heap root.  A new tile has a lower id than every
@@ -153,6 +155,58 @@ MSA_DEV void write_selection(const uint2* heap, int k1, int topk, int dil, int q
                 if (slot < topk) out[slot] = v[w];
             }
             if (lane == 0) nsel[row0 + row] = topk;
+        }
+    }
+}
+
+// Ascending sort of N ints held by one thread (bitonic network, fully
+// unrolled: every index is a compile-time constant, so v stays in registers).
+template <int N>
+MSA_DEV void thread_sort(int (&v)[N])
+{
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const int a = v[i], b = v[l];
+                    const bool up = (i & k) == 0;
+                    v[i] = up ? min(a, b) : max(a, b);
+                    v[l] = up ? max(a, b) : min(a, b);
+                }
+            }
+        }
+    }
+}
+
+// The warp's 32 rows (TMEM lane quarter q), topk <= N: every thread sorts
+// its own row's k1 kept ids and the topk - k1 forced blocks in registers (all
+// 32 rows at once, no shuffles), parks the result in shared memory ([row][N+1]
+// ints: the odd row stride keeps both access patterns free of bank
+// conflicts) and the warp writes the rows out coalesced.
+template <int N>
+MSA_DEV void write_selection_rows(const uint2* heap, int k1, int topk, int dil, int q, int qb, int T, int64_t row0,
+                                  int32_t* idx, int32_t* nsel, int32_t* stg)
+{
+    const int lane = (int)(threadIdx.x & 31u);
+    const int row = q * 32 + lane;
+    int v[N];
+#pragma unroll
+    for (int s = 0; s < N; ++s)
+        v[s] = s < k1 ? (int)heap[s * 128 + row].y : (s < topk ? qb - (s - k1) * dil : 0x7fffffff);
+    thread_sort<N>(v);
+#pragma unroll
+    for (int s = 0; s < N; ++s) stg[row * (N + 1) + s] = v[s];
+    __syncwarp();
+    for (int rr = 0; rr < 32; ++rr) {
+        const int r2 = q * 32 + rr;
+        if (qb * 128 + r2 < T) {   // warp-uniform
+            int32_t* out = idx + (row0 + r2) * topk;
+            for (int s = lane; s < topk; s += 32) out[s] = stg[r2 * (N + 1) + s];
+            if (lane == 0) nsel[row0 + r2] = topk;
         }
     }
 }
@@ -405,9 +459,16 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
         __syncwarp();   // each lane's heap column is read by the whole warp below
         if (go) {
             if (need_heap) {
+                // every MMA has finished (the last pair's maxima have been
+                // read), so the key ring is free to stage the sorted rows
                 const int64_t row0 = (int64_t)bg * p.T + qb * 128;
-                if (p.topk <= 64)
-                    write_selection<2>(heap, k1, p.topk, p.dilation, warp - 10, qb, p.T, row0, p.idx, p.nsel);
+                int32_t* stg = (int32_t*)kp_tiles;
+                if (p.topk <= 32)
+                    write_selection_rows<32>(heap, k1, p.topk, p.dilation, warp - 10, qb, p.T, row0, p.idx, p.nsel,
+                                             stg);
+                else if (p.topk <= 64)
+                    write_selection_rows<64>(heap, k1, p.topk, p.dilation, warp - 10, qb, p.T, row0, p.idx, p.nsel,
+                                             stg);
                 else
                     write_selection<4>(heap, k1, p.topk, p.dilation, warp - 10, qb, p.T, row0, p.idx, p.nsel);
             } else if (row_ok) {

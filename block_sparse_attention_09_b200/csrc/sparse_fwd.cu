@@ -6,14 +6,18 @@
 // Sparse Attention Kernels Debut", section "How MSA works": GQA main
 // attention, block ids cached by the Index Branch).
 //
-// KV-stationary design.  One CTA owns one KV block n of one group: its K and
-// V tiles (128 keys) are loaded once by TMA; the queries that selected the
-// block are gathered from the inverse index in chunks of 128 rows (128/G
-// tokens x the G query heads of the group, head-major: row = hh * 128/G + t)
-// with cp.async into a 3-stage ring.
-// Per chunk:  S = Q K^T (tcgen05, TMEM) -> P = exp2(S*scale*log2e - m_i) written
-// back to TMEM as bf16 -> O_part = P V (tcgen05 with A from TMEM) -> fp32
-// reductions of O_part and of the row sums into global accumulators.
+// KV-stationary design over PAIRS of KV blocks.  One CTA owns the blocks 2p
+// and 2p+1 of one group: their K and V tiles (2 x 128 keys) are loaded once by
+// TMA; the queries that selected either block are gathered from the pair
+// index in chunks of 128 rows (128/G tokens x the G query heads of the group,
+// head-major: row = hh * 128/G + t) with cp.async into a 2-stage ring.
+// Per chunk and block:  S = Q K^T (tcgen05, TMEM) -> P = exp2(S*scale*log2e -
+// m_i), zero for a block the row did not select, written back to TMEM as
+// bf16 -> O_part += P V (tcgen05 with A from TMEM); then fp32 reductions of
+// O_part and of the row sums into global accumulators.  The main cost of a
+// KV-stationary forward is on-chip traffic per (row, block) pair -- the query
+// gather and the fp32 O reduction -- and a row that selected both blocks of a
+// pair pays it once: with selections that favour nearby blocks most rows do.
 //
 // Softmax normalisation across the CTAs that share a query row uses a fixed
 // per-row shift m_i instead of a running maximum, so every CTA's partial sums
@@ -41,38 +45,63 @@ namespace msa {
 namespace {
 
 constexpr int kThreads = 448;   // w0 TMA(K,V) | w1 MMA | w2-5 gather | w6-9 softmax | w10-13 O out
-constexpr int kQStages = 3;
+constexpr int kQStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSumLow = 7.703719777548943e-34f;     // 2^-110: row sums outside [kSumLow, kSumHigh]
 constexpr float kSumHigh = 1.2676506002282294e30f;    // 2^100   (or not finite) are redone exactly
 constexpr float kShiftSlack = 100.f;                  // m_i <= S_ii + kShiftSlack (log2 units)
 
 struct FwdParams {
-    int B, T, Hq, Hkv, lgG, tpc, nblk, topk;
+    int B, T, Hq, Hkv, lgG, tpc, nblk, npair, topk;
     int RB, qb0, per_group;   // query blocks per range; first query block; work items per (b, group)
     float c1;        // scale * log2(e)
     const __nv_bfloat16* q;
-    const int32_t* ptr;
-    const int32_t* off;
-    const int32_t* tok;
-    const float* shift;   // m_i per [b][h][i], log2 units
+    const int32_t* ptr2;
+    const int32_t* off2;
+    const int32_t* tok2;   // pair lists: (i << 2) | selected 2p | selected 2p+1 << 1
+    const float* shift;    // m_i per [b][h][i], log2 units
     float* oacc;
     float* lacc;
+    float* bmass;          // nullable: per pair-list entry [e][2][G], the row's weight sum of each block
     uint32_t* status;
 };
 
 template <int D>
+struct FwdSmem {
+    static constexpr uint32_t kTile = 128u * D * 2u;                 // 128 rows x D bf16
+    static constexpr uint32_t kKV = 0;                               // K0, V0, K1, V1
+    static constexpr uint32_t kQ = 4 * kTile;                        // kQStages query chunks
+    static constexpr uint32_t kStg = kQ + kQStages * kTile;          // O staging: half a chunk's tokens
+    static constexpr uint32_t kStgBytes = 64u * D * 4u + 1024u;      // 64 rows of D fp32 + 16 B per token
+    static constexpr uint32_t kBars = kStg + kStgBytes;
+    static constexpr uint32_t kTotal = kBars + 32 * 8 + 16;
+    static_assert(kTotal <= 232448, "shared memory per CTA");
+};
+
+// One CTA per work item: a pair of KV blocks n0 = 2p, n1 = 2p+1 of one group
+// and the queries of one range that selected either.  Chunk c holds 128 rows
+// (128/G tokens x the G heads, head-major); per chunk and sub-block s:
+//   S_s = Q K_s^T -> TMEM [128 s, 128 s + 128)
+//   P_s = exp2(S_s c1 - m_i), zero where the row did not select block n_s or
+//         the key is after the query, written back over S_s as bf16
+//   O  += P_s V_s (A from TMEM) into one of two O buffers
+// so that a row that selected both blocks is gathered once and adds one O
+// partial for both.
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                FwdParams p)
+fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, FwdParams p)
 {
-    constexpr uint32_t kTile = 128u * D * 2u;   // 128 rows x D bf16
+    using SM = FwdSmem<D>;
+    constexpr uint32_t kTile = SM::kTile;
     constexpr int kSlabs = D / 64;
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const RangeItem item = range_item((int)blockIdx.x, p.nblk, p.RB, p.qb0, p.per_group, p.ptr, p.off);
-    const int n = item.n, bg = item.bg;
+    int qe = 0;
+    const RangeItem item = pair_item((int)blockIdx.x, p.nblk, p.npair, p.RB, p.qb0, p.per_group, p.ptr2, p.off2, &qe);
+    const int pn = item.n, bg = item.bg;
+    const int n0 = 2 * pn, n1 = 2 * pn + 1;
+    const int nsub = n1 < qe ? 2 : 1;   // block n1 is read by a query of this range only if n1 < qe
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int G = 1 << p.lgG;
     const int count = item.count;
@@ -82,25 +111,25 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (threadIdx.x == 0) atomicCAS(p.status, 0u, code0 + 15);
         return;
     }
-    const int32_t* toks = p.tok + (int64_t)bg * p.T * p.topk + item.beg;
+    const int32_t* toks = p.tok2 + (int64_t)bg * p.T * p.topk + item.beg;
     const int nchunks = (count + p.tpc - 1) / p.tpc;
 
-    uint8_t* k_tile = smem;
-    uint8_t* v_tile = smem + kTile;
-    uint8_t* q_st = smem + 2 * kTile;
-    // O staging: token t of a chunk at t * (G*D*4 + 16) bytes; the 16-byte pad
-    // per token spreads the rows of a warp over all banks.
-    uint8_t* o_stg = q_st + kQStages * kTile;
+    auto k_tile = [&](int s) { return smem + SM::kKV + (uint32_t)(2 * s) * kTile; };
+    auto v_tile = [&](int s) { return smem + SM::kKV + (uint32_t)(2 * s + 1) * kTile; };
+    uint8_t* q_st = smem + SM::kQ;
+    // O staging of half a chunk's tokens: token t' at t' * (G*D*4 + 16) bytes;
+    // the 16-byte pad per token spreads the rows of a warp over all banks.
+    uint8_t* o_stg = smem + SM::kStg;
     const uint32_t tok_bytes = (uint32_t)G * D * 4u;
     const uint32_t tok_stride = tok_bytes + 16u;
-    uint64_t* bars = (uint64_t*)(o_stg + 128 * D * 4 + 2048);
+    uint64_t* bars = (uint64_t*)(smem + SM::kBars);
     uint64_t* kv_full = bars;
-    uint64_t* q_full = bars + 1;
-    uint64_t* q_empty = q_full + kQStages;
-    uint64_t* s_full = q_empty + kQStages;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* o_full = p_full + 2;
-    uint64_t* o_empty = o_full + 2;
+    uint64_t* q_full = bars + 1;                 // [kQStages]
+    uint64_t* q_empty = q_full + kQStages;       // [kQStages]
+    uint64_t* s_full = q_empty + kQStages;       // [2] per sub-block
+    uint64_t* p_full = s_full + 2;               // [2] per sub-block
+    uint64_t* o_full = p_full + 2;               // [2] per O buffer
+    uint64_t* o_empty = o_full + 2;              // [2] per O buffer
     uint64_t* fin = o_empty + 2;
     uint32_t* tmem_hold = (uint32_t*)(fin + 1);
     volatile uint32_t* abort_flag = tmem_hold + 1;
@@ -124,18 +153,19 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_hold;
-    // TMEM columns: S/P buffers at 0 and 128, O buffers at 256 and 256 + D.
+    // TMEM columns: S/P of sub-block s at 128 s, O buffers at 256 and 256 + D.
 
     if (warp == 0) {
-        // ---------------- K/V tiles (once) ----------------
+        // ---------------- K/V tiles of both blocks (once) ----------------
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(kv_full, 2 * kTile);
-            for (int s = 0; s < kSlabs; ++s) {
-                tma_load_4d(k_tile + s * 16384, &tm_k, kv_full, s * 64, g, n * 128, b);
-                tma_load_4d(v_tile + s * 16384, &tm_v, kv_full, s * 64, g, n * 128, b);
-            }
+            mbar_arrive_expect_tx(kv_full, 2u * nsub * kTile);
+            for (int s = 0; s < nsub; ++s)
+                for (int sl = 0; sl < kSlabs; ++sl) {
+                    tma_load_4d(k_tile(s) + sl * 16384, &tm_k, kv_full, sl * 64, g, (n0 + s) * 128, b);
+                    tma_load_4d(v_tile(s) + sl * 16384, &tm_v, kv_full, sl * 64, g, (n0 + s) * 128, b);
+                }
             mbar_drain(kv_full, 0);   // the tiles must have landed before this warp leaves
         }
     } else if (warp == 1) {
@@ -143,40 +173,50 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idPV = idesc_bf16(128, D, false, true);
-            const uint32_t ka = smem_u32(k_tile), va = smem_u32(v_tile), qa = smem_u32(q_st);
-            // S(c+2) reuses the TMEM columns where P(c) lives, so it is issued
-            // only after every K-step of PV(c) (MMAs of one thread run in order).
-            auto issue_s = [&](int c) -> bool {
-                const int s = c % kQStages;
-                const uint32_t use = (uint32_t)(c / kQStages);
-                if (!mbar_wait(&q_full[s], use & 1u, wc, code0 + 1)) return false;
-                tc_fence_after();
-                const uint32_t qs = qa + s * kTile;
-                const uint32_t dS = tmem + (uint32_t)(c & 1) * 128u;
+            const uint32_t qa = smem_u32(q_st);
+            // S(c, s) into the columns of sub-block s.  A sub-block's columns
+            // still hold P of the previous chunk until its PV MMAs have run, so
+            // S(c, s) is issued after PV(c-1, s) (MMAs of one thread run in order).
+            auto issue_s = [&](int c, int s) {
+                const uint32_t qs = qa + (uint32_t)(c % kQStages) * kTile;
+                const uint32_t ka = smem_u32(k_tile(s));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(dS, desc_kmajor(qs, 128, kk * 16), desc_kmajor(ka, 128, kk * 16), idS,
-                            kk > 0 ? 1u : 0u);
-                umma_commit(&q_empty[s]);
-                umma_commit(&s_full[c & 1]);
-                return true;
+                    umma_ss(tmem + (uint32_t)s * 128u, desc_kmajor(qs, 128, kk * 16), desc_kmajor(ka, 128, kk * 16),
+                            idS, kk > 0 ? 1u : 0u);
+                umma_commit(&s_full[s]);
+                if (s == nsub - 1) umma_commit(&q_empty[c % kQStages]);   // the chunk's queries are read
+            };
+            auto wait_q = [&](int c) {
+                return mbar_wait(&q_full[c % kQStages], (uint32_t)(c / kQStages) & 1u, wc, code0 + 1);
             };
             bool ok = mbar_wait(kv_full, 0, wc, code0 + 0);
-            if (ok && nchunks > 0) ok = issue_s(0);
-            if (ok && nchunks > 1) ok = issue_s(1);
+            if (ok && nchunks > 0) {
+                ok = wait_q(0);
+                if (ok) {
+                    tc_fence_after();
+                    for (int s = 0; s < nsub; ++s) issue_s(0, s);
+                }
+            }
             for (int c = 0; ok && c < nchunks; ++c) {
                 const int buf = c & 1;
                 const uint32_t use = (uint32_t)(c >> 1);
-                if (!mbar_wait(&p_full[buf], use & 1u, wc, code0 + 2)) break;
-                if (use > 0 && !mbar_wait(&o_empty[buf], (use - 1) & 1u, wc, code0 + 3)) break;
-                tc_fence_after();
-                const uint32_t pa = tmem + (uint32_t)buf * 128u;
                 const uint32_t oa = tmem + 256u + (uint32_t)buf * D;
+                if (use > 0 && !mbar_wait(&o_empty[buf], (use - 1) & 1u, wc, code0 + 3)) break;
+                for (int s = 0; ok && s < nsub; ++s) {
+                    if (!mbar_wait(&p_full[s], (uint32_t)c & 1u, wc, code0 + 2)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t pa = tmem + (uint32_t)s * 128u, va = smem_u32(v_tile(s));
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(oa, pa + kk * 8, desc_mnmajor(va, 128, kk * 16), idPV, kk > 0 ? 1u : 0u);
-                umma_commit(&o_full[buf]);
-                if (c + 2 < nchunks) ok = issue_s(c + 2);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ts(oa, pa + kk * 8, desc_mnmajor(va, 128, kk * 16), idPV, (s > 0 || kk > 0) ? 1u : 0u);
+                    if (s == nsub - 1) umma_commit(&o_full[buf]);
+                    if (c + 1 < nchunks) {
+                        if (s == 0 && !wait_q(c + 1)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_s(c + 1, s);
+                    }
+                }
             }
             umma_commit(fin);
             mbar_drain(fin, 0);
@@ -198,7 +238,7 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const int t = row & (p.tpc - 1), hh = row >> (7 - p.lgG);
                 const int jj = c * p.tpc + t;
                 const bool valid = jj < count;
-                const int i = valid ? toks[jj] : 0;
+                const int i = valid ? (toks[jj] >> 2) : 0;
                 const __nv_bfloat16* src =
                     p.q + (((int64_t)b * p.T + i) * p.Hq + g * G + hh) * D + ch * 8;
                 cp_async_16(qs + sw128_offset(row, ch & 7, ch >> 3, 128), src, valid ? 16u : 0u);
@@ -215,100 +255,122 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
         const int t = r & (p.tpc - 1), hh = r >> (7 - p.lgG), h = g * G + hh;
         const float* shift_row = p.shift + ((int64_t)b * p.Hq + h) * p.T;
-        // this row's token and shift are loaded one and two chunks ahead, so
+        // this row's entry and shift are loaded one and two chunks ahead, so
         // the dependent global loads overlap the previous chunk's work
-        auto tok_of = [&](int cc) { const int jj = cc * p.tpc + t; return jj < count ? toks[jj] : -1; };
-        int tok_cur = tok_of(0), tok_nxt = nchunks > 1 ? tok_of(1) : -1;
-        float sh_cur = tok_cur >= 0 ? shift_row[tok_cur] : 0.f;
+        auto ent_of = [&](int cc) { const int jj = cc * p.tpc + t; return jj < count ? toks[jj] : -1; };
+        int ent_cur = ent_of(0), ent_nxt = nchunks > 1 ? ent_of(1) : -1;
+        float sh_cur = ent_cur >= 0 ? shift_row[ent_cur >> 2] : 0.f;
         for (int c = 0; c < nchunks; ++c) {
-            const int buf = c & 1;
-            const uint32_t use = (uint32_t)(c >> 1);
-            const int tok_nn = c + 2 < nchunks ? tok_of(c + 2) : -1;
-            const float sh_nxt = tok_nxt >= 0 ? shift_row[tok_nxt] : 0.f;
-            const bool ok = mbar_wait(&s_full[buf], use & 1u, wc, code0 + 5);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-            const bool valid = tok_cur >= 0;
-            const int i = valid ? tok_cur : 0;
-            const int cmax = valid ? (((i >> 7) == n) ? (i & 127) : 127) : -1;
+            const int ent_nn = c + 2 < nchunks ? ent_of(c + 2) : -1;
+            const float sh_nxt = ent_nxt >= 0 ? shift_row[ent_nxt >> 2] : 0.f;
+            const bool valid = ent_cur >= 0;
+            const int i = valid ? (ent_cur >> 2) : 0;
             const float mh = valid ? sh_cur : 0.f;
-            tok_cur = tok_nxt;
-            tok_nxt = tok_nn;
+            const int flags = valid ? (ent_cur & 3) : 0;
+            ent_cur = ent_nxt;
+            ent_nxt = ent_nn;
             sh_cur = sh_nxt;
-            const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)buf * 128u);
             float l = 0.f;
+            bool ok = true;
+            const int64_t ent_idx = (int64_t)bg * p.T * p.topk + item.beg + c * p.tpc + t;   // this row's entry
+            for (int s = 0; s < nsub; ++s) {
+                float ls = 0.f;
+                ok = mbar_wait(&s_full[s], (uint32_t)c & 1u, wc, code0 + 5);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                // last key of block n0 + s this row reads (-1: none)
+                const int cmax = !((flags >> s) & 1) ? -1 : (((i >> 7) == n0 + s) ? (i & 127) : 127);
+                const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)s * 128u);
 #pragma unroll
-            for (int piece = 0; piece < 4; ++piece) {
-                uint32_t v[32], pk[16];
-                tmem_ld32(ta + piece * 32, v);
-                tmem_ld_wait();
+                for (int piece = 0; piece < 4; ++piece) {
+                    uint32_t v[32], pk[16];
+                    tmem_ld32(ta + piece * 32, v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int c0 = piece * 32 + 2 * e;
-                    const float p0 = c0 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e]), p.c1, -mh)) : 0.f;
-                    const float p1 = c0 + 1 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mh)) : 0.f;
-                    pk[e] = pack_bf16x2(p0, p1);
-                    // normalise by the weights the PV product actually uses (bf16), so
-                    // that O is an exact convex combination of the selected values
-                    l += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+                    for (int e = 0; e < 16; ++e) {
+                        const int c0 = piece * 32 + 2 * e;
+                        const float p0 = c0 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e]), p.c1, -mh)) : 0.f;
+                        const float p1 = c0 + 1 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mh)) : 0.f;
+                        pk[e] = pack_bf16x2(p0, p1);
+                        // normalise by the weights the PV product actually uses (bf16), so
+                        // that O is an exact convex combination of the selected values
+                        ls += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+                    }
+                    tmem_st16(ta + piece * 16, pk);   // P overwrites S columns already read
                 }
-                tmem_st16(ta + piece * 16, pk);   // P overwrites S columns already read
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&p_full[s]);
+                l += ls;
+                if (p.bmass != nullptr && ((flags >> s) & 1)) p.bmass[(ent_idx * 2 + s) * G + hh] = ls;
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&p_full[buf]);
+            if (!ok) break;
             if (valid) atomicAdd(&p.lacc[((int64_t)b * p.Hq + h) * p.T + i], l);
         }
     } else {
         // ---------------- O partials -> fp32 global accumulators ----------------
         // TMEM -> padded staging in shared memory -> one bulk fp32 reduction of
         // G*D floats per token (whole cache lines at L2 instead of 16-byte
-        // reductions from every thread).  Rows are head-major, so the eight
-        // lanes of one 16-byte store phase hold eight different tokens and the
-        // per-token pad puts them on eight different bank groups.
+        // reductions from every thread).  The staging holds half a chunk's
+        // tokens, so each chunk goes out in two halves.  Rows are head-major,
+        // so the eight lanes of one 16-byte store phase hold eight different
+        // tokens and the per-token pad puts them on eight different bank groups.
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
         const int t = r & (p.tpc - 1), hh = r >> (7 - p.lgG);
-        const int tid = threadIdx.x - 320;             // token this thread reduces
+        const int half_tok = p.tpc >> 1;                       // tokens per half
+        const int my_half = t >= half_tok ? 1 : 0;
+        const int tid = threadIdx.x - 320;                     // token (within a half) this thread reduces
         const uint32_t stg = smem_u32(o_stg);
-        const uint32_t my_row = stg + (uint32_t)t * tok_stride + (uint32_t)hh * D * 4u;
-        int my_tok_id = tid < min(p.tpc, count) ? toks[tid] : 0;
+        const uint32_t my_row = stg + (uint32_t)(t - my_half * half_tok) * tok_stride + (uint32_t)hh * D * 4u;
+        auto tok_at = [&](int cc, int hf) {
+            const int jj = cc * p.tpc + hf * half_tok + tid;
+            return (cc < nchunks && tid < half_tok && jj < count) ? (toks[jj] >> 2) : -1;
+        };
+        int tk0 = tok_at(0, 0), tk1 = tok_at(0, 1);
         bool issued = false;
-        for (int c = 0; c < nchunks; ++c) {
+        bool ok = true;
+        for (int c = 0; c < nchunks && ok; ++c) {
             const int buf = c & 1;
             const uint32_t use = (uint32_t)(c >> 1);
-            const bool ok = mbar_wait(&o_full[buf], use & 1u, wc, code0 + 6);
-            // the previous chunk's bulk reductions must have read the staging
-            if (issued) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-            if (!bar_and_sync(2, 128, ok)) break;   // all four warps go on, or none
-            tc_fence_after();
-            const uint32_t ta = tmem_addr(tmem, lane_base, 256u + (uint32_t)buf * D);
+            ok = mbar_wait(&o_full[buf], use & 1u, wc, code0 + 6);
+            const int nt0 = tk0, nt1 = tk1;
+            tk0 = tok_at(c + 1, 0);   // next chunk's, loaded early
+            tk1 = tok_at(c + 1, 1);
+            for (int hf = 0; hf < 2; ++hf) {
+                // the previous half's bulk reductions must have read the staging
+                if (issued) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                if (!bar_and_sync(2, 128, ok)) { ok = false; break; }   // all four warps go on, or none
+                tc_fence_after();
+                const uint32_t ta = tmem_addr(tmem, lane_base, 256u + (uint32_t)buf * D);
 #pragma unroll
-            for (int piece = 0; piece < D / 32; ++piece) {
-                uint32_t v[32];
-                tmem_ld32(ta + piece * 32, v);
-                tmem_ld_wait();
+                for (int piece = 0; piece < D / 32; ++piece) {
+                    uint32_t v[32];
+                    tmem_ld32(ta + piece * 32, v);
+                    tmem_ld_wait();
+                    if (my_half == hf) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + (piece * 32 + 4 * e) * 4),
-                                 "r"(v[4 * e]), "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3])
+                        for (int e = 0; e < 8; ++e)
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + (piece * 32 + 4 * e) * 4),
+                                         "r"(v[4 * e]), "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3])
+                                         : "memory");
+                    }
+                }
+                if (hf == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&o_empty[buf]);     // the TMEM buffer is free once copied out
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(2, 128);
+                const int i = hf == 0 ? nt0 : nt1;
+                issued = i >= 0;
+                if (issued) {
+                    float* dst = p.oacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D;
+                    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+                                 "r"(stg + (uint32_t)tid * tok_stride), "r"(tok_bytes)
                                  : "memory");
-            }
-            tc_fence_before();
-            mbar_arrive(&o_empty[buf]);     // the TMEM buffer is free once copied out
-            fence_proxy_async_smem();
-            named_bar_sync(2, 128);
-            const int ntok = min(p.tpc, count - c * p.tpc);
-            const int i = my_tok_id;
-            my_tok_id = (c + 1 < nchunks && tid < p.tpc && (c + 1) * p.tpc + tid < count)
-                            ? toks[(c + 1) * p.tpc + tid] : 0;   // next chunk's, loaded early
-            issued = tid < ntok;
-            if (issued) {
-                float* dst = p.oacc + (((int64_t)b * p.T + i) * p.Hq + g * G) * D;
-                asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
-                             "r"(stg + (uint32_t)tid * tok_stride), "r"(tok_bytes)
-                             : "memory");
-                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
             }
         }
         // the staging must have been read before the CTA exits; the global
@@ -545,7 +607,7 @@ template <int D>
 cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const void* v,
                          const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int32_t* idx,
                          const int32_t* nsel, void* o, float* lse, void* ws, const WsLayout& L,
-                         cudaStream_t st)
+                         float* bmass, cudaStream_t st)
 {
     uint8_t* w = (uint8_t*)ws;
     float* shift = (float*)(w + L.shift);
@@ -572,18 +634,18 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     FwdParams p;
     p.B = pr.B; p.T = pr.T; p.Hq = pr.Hq; p.Hkv = pr.Hkv;
     p.lgG = 31 - __builtin_clz((unsigned)pr.G);
-    p.tpc = 128 / pr.G; p.nblk = pr.nblk; p.topk = pr.topk;
+    p.tpc = 128 / pr.G; p.nblk = pr.nblk; p.npair = pair_count(pr.nblk); p.topk = pr.topk;
     p.c1 = c1;
     p.q = qb;
-    p.ptr = (const int32_t*)(w + L.ptr);
-    p.off = (const int32_t*)(w + L.cnt);
-    p.tok = (const int32_t*)(w + L.tok);
-    p.shift = shift; p.oacc = oacc; p.lacc = lacc;
+    p.ptr2 = (const int32_t*)(w + L.ptr2);
+    p.off2 = (const int32_t*)(w + L.cnt2);
+    p.tok2 = (const int32_t*)(w + L.tok2);
+    p.shift = shift; p.oacc = oacc; p.lacc = lacc; p.bmass = bmass;
     p.status = (uint32_t*)(w + L.status);
     p.RB = range_blocks(pr);
     p.qb0 = pr.qb0;
-    p.per_group = range_items_per_group(pr.nblk, p.RB, pr.qb0);
-    const size_t smem = (size_t)(2 + kQStages) * 128 * D * 2 + 128 * D * 4 + 2048 + 32 * 8;
+    p.per_group = pair_items_per_group(pr.nblk, p.RB, pr.qb0);
+    const size_t smem = FwdSmem<D>::kTotal;
     if ((e = cudaFuncSetAttribute(fwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
         return e;
@@ -608,10 +670,10 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
 cudaError_t launch_fwd(const Problem& pr, const void* q, const void* k, const void* v,
                        const CUtensorMap& tm_k, const CUtensorMap& tm_v, const int32_t* idx,
                        const int32_t* nsel, void* o, float* lse, void* ws, const WsLayout& L,
-                       cudaStream_t st)
+                       float* bmass, cudaStream_t st)
 {
-    if (pr.d == 64) return launch_fwd_d<64>(pr, q, k, v, tm_k, tm_v, idx, nsel, o, lse, ws, L, st);
-    return launch_fwd_d<128>(pr, q, k, v, tm_k, tm_v, idx, nsel, o, lse, ws, L, st);
+    if (pr.d == 64) return launch_fwd_d<64>(pr, q, k, v, tm_k, tm_v, idx, nsel, o, lse, ws, L, bmass, st);
+    return launch_fwd_d<128>(pr, q, k, v, tm_k, tm_v, idx, nsel, o, lse, ws, L, bmass, st);
 }
 
 }  // namespace msa

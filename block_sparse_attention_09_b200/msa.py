@@ -24,8 +24,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
-MSA_SELECT, MSA_FWD, MSA_BWD, MSA_DECODE = 0, 1, 2, 3
-MSA_REUSE_INDEX, MSA_DKV_F32 = 1, 2
+MSA_SELECT, MSA_FWD, MSA_BWD, MSA_DECODE, MSA_PROXY_BWD = 0, 1, 2, 3, 4
+MSA_REUSE_INDEX, MSA_DKV_F32, MSA_BLOCK_MASS = 1, 2, 4
 _ERR = {0: "ok", -1: "invalid dimensions", -2: "null pointer", -3: "misaligned pointer",
         -4: "workspace too small", -5: "CUDA launch failed", -6: "device wait timed out",
         -7: "device is not sm_100", -8: "tensor map encoding failed",
@@ -70,6 +70,8 @@ def _load():
     lib.msa_decode.restype = I
     lib.msa_f32_to_bf16.argtypes = [P, P, ctypes.c_int64, P]
     lib.msa_f32_to_bf16.restype = I
+    lib.msa_proxy_bwd.argtypes = [D, P, P, P, P, P, P, P, P, SZ, P]
+    lib.msa_proxy_bwd.restype = I
     lib.msa_fallback_rows.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     lib.msa_fallback_rows.restype = I
     lib.msa_kernel_launches.argtypes = []
@@ -166,9 +168,11 @@ def proxy_select(qp, kp, topk, pooled=False, stream=None, ws=None, check=False, 
 
 
 def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=None, reuse_index=False,
-        q_begin=0):
+        q_begin=0, block_mass=False):
     """Main Branch forward.  Returns (o bf16 [B,T,Hq,d], lse fp32 [B,Hq,T]).
-    q_begin: first query row computed; earlier rows of o, lse are unwritten."""
+    q_begin: first query row computed; earlier rows of o, lse are unwritten.
+    block_mass: also keep each row's weight per selected block in ``ws`` (a
+    proxy_workspace) for a following proxy_bwd."""
     _bf16(q, k, v)
     B, T, Hq, d = q.shape
     topk = idx.shape[3]
@@ -179,9 +183,10 @@ def fwd(q, k, v, idx, nsel, scale=0.0, stream=None, ws=None, check=False, out=No
     else:
         o, lse = out
     if ws is None:
-        ws = workspace(dims, MSA_FWD, q.device)
+        ws = workspace(dims, MSA_PROXY_BWD if block_mass else MSA_FWD, q.device)
+    flags = (MSA_REUSE_INDEX if reuse_index else 0) | (MSA_BLOCK_MASS if block_mass else 0)
     _check(LIB.msa_fwd_ex(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(idx), _p(nsel), _p(o), _p(lse), _p(ws),
-                          ws.numel(), _stream(stream), MSA_REUSE_INDEX if reuse_index else 0), "msa_fwd")
+                          ws.numel(), _stream(stream), flags), "msa_fwd")
     if check:
         _check(check_status(ws, stream), "msa_fwd (device)")
     return o, lse
@@ -214,6 +219,33 @@ def bwd(q, k, v, o, dout, lse, idx, nsel, scale=0.0, stream=None, ws=None, check
     if check:
         _check(check_status(ws, stream), "msa_bwd (device)")
     return dq, dk, dv
+
+
+def proxy_workspace(dims: Dims, device) -> torch.Tensor:
+    """One workspace for a forward that keeps block masses, the backward
+    that reuses its index, and the proxy-head gradient."""
+    return torch.empty(max(workspace_size(dims, MSA_PROXY_BWD), 256), dtype=torch.uint8, device=device)
+
+
+def proxy_bwd(q, qp, kp, idx, nsel, ws, stream=None, check=False, out=None, q_begin=0):
+    """Proxy-head gradient (a KL distillation of the Main Branch's block
+    weights into the proxy scores; see include/msa.h).  ``ws`` must hold what
+    fwd(..., block_mass=True) left for these idx/nsel.  Returns (dqp, dkp fp32
+    [B,T,Hp,dp], loss fp32 [B,Hp,T])."""
+    _bf16(qp, kp)
+    B, T, Hp, dp = qp.shape
+    dims = make_dims(B, T, q.shape[2], Hp, q.shape[3], dp, idx.shape[3], q_begin=q_begin)
+    if out is None:
+        dqp = torch.zeros(qp.shape, dtype=torch.float32, device=qp.device)
+        dkp = torch.empty(kp.shape, dtype=torch.float32, device=kp.device)
+        loss = torch.zeros((B, Hp, T), dtype=torch.float32, device=qp.device)
+    else:
+        dqp, dkp, loss = out
+    _check(LIB.msa_proxy_bwd(ctypes.byref(dims), _p(qp), _p(kp), _p(idx), _p(nsel), _p(dqp), _p(dkp), _p(loss),
+                             _p(ws), ws.numel(), _stream(stream)), "msa_proxy_bwd")
+    if check:
+        _check(check_status(ws, stream), "msa_proxy_bwd (device)")
+    return dqp, dkp, loss
 
 
 def f32_to_bf16(src, out=None, stream=None):

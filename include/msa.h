@@ -91,7 +91,7 @@ enum msa_status {
     MSA_ERR_INDEX = -9          /* an idx entry outside its valid range       */
 };
 
-enum msa_phase { MSA_SELECT = 0, MSA_FWD = 1, MSA_BWD = 2, MSA_DECODE = 3 };
+enum msa_phase { MSA_SELECT = 0, MSA_FWD = 1, MSA_BWD = 2, MSA_DECODE = 3, MSA_PROXY_BWD = 4 };
 
 /* Bytes of workspace `which` (an msa_phase) needs for these dims.
  * Returns 0 for invalid dims. */
@@ -210,7 +210,14 @@ MSA_API int msa_decode(const msa_dims* dims, const int32_t* lens, const void* q,
  * Reusing an index built from different idx is undefined.  flags = 0 is
  * msa_fwd / msa_bwd.
  */
-enum msa_flags { MSA_REUSE_INDEX = 1, MSA_DKV_F32 = 2 };
+enum msa_flags { MSA_REUSE_INDEX = 1, MSA_DKV_F32 = 2, MSA_BLOCK_MASS = 4 };
+/* MSA_BLOCK_MASS (msa_fwd_ex): the forward also keeps, in `ws`, the softmax
+ * weight each query row puts on each of its selected blocks, for a following
+ * msa_proxy_bwd on the same workspace.  `ws` must then hold
+ * msa_workspace_size(dims, MSA_PROXY_BWD) bytes; that layout keeps the
+ * forward's and the backward's regions at their usual offsets, so one such
+ * workspace serves msa_fwd_ex, msa_bwd_ex (MSA_REUSE_INDEX) and
+ * msa_proxy_bwd of one step. */
 /* MSA_DKV_F32 (msa_bwd_ex): dk and dv are fp32 [B][T][Hkv][d] and receive the
  * unrounded sums, so that partial gradients of several query shards can be
  * added (a reduce-scatter) before one rounding to bf16 (msa_f32_to_bf16). */
@@ -219,6 +226,34 @@ MSA_API int msa_fwd_ex(const msa_dims* dims, const void* q, const void* k, const
 MSA_API int msa_bwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v, const void* o,
                        const void* dout, const float* lse, const int32_t* idx, const int32_t* nsel, void* dq,
                        void* dk, void* dv, void* ws, size_t ws_bytes, void* stream, int flags);
+
+/*
+ * Proxy-head gradient (the ai-beat post on Flash-MSA training, paragraph 2:
+ * gradients through the gating mechanism; paragraph 4: the proxy heads are
+ * trained).  The pages do not define the training signal; this entry point
+ * computes one reading of it, the KL divergence that distils the Main
+ * Branch's attention into the Index Branch (as DeepSeek's indexer is trained,
+ * which "How MSA works" likens MSA to).  Per query row (b, g, i) over its
+ * selected blocks S (idx, nsel):
+ *   p(n) = (1/G) sum over the group's heads of the softmax weight the
+ *          forward put on the keys of block n (held constant),
+ *   z(n) = the pooled proxy score of block n (max over its keys j <= i),
+ *   q    = softmax over S of z,   loss[b][g][i] = KL(p || q),
+ * and with dz(n) = q(n) sum_m p(m) - p(n) and j*(n) the argmax key of block
+ * n (the lowest key on ties), dqp_i = sum_n dz(n) kp_j*(n),
+ * dkp_j = sum over (i, n) with j*(n) = j of dz(n) qp_i.
+ *   dqp [B][T][Hp][dp] fp32 (rows q_begin .. T-1 written), dkp
+ *   [B][T][Hp][dp] fp32 (every row written), loss [B][Hp][T] fp32 (rows
+ *   q_begin .. T-1).
+ * `ws` (msa_workspace_size(dims, MSA_PROXY_BWD) bytes) must hold what an
+ * earlier msa_fwd_ex with MSA_BLOCK_MASS left there for exactly these dims,
+ * idx and nsel; a msa_bwd_ex on the same workspace in between is allowed.
+ * A row whose forward weights overflowed (only rows the exact fallback redid,
+ * msa_fallback_rows, can) gets loss 0 and no gradient.
+ */
+MSA_API int msa_proxy_bwd(const msa_dims* dims, const void* qp, const void* kp, const int32_t* idx,
+                          const int32_t* nsel, float* dqp, float* dkp, float* loss, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* dst[i] = bf16(src[i]) (round to nearest even) for i < n: fp32 -> bf16 on
  * the device.  n must be a multiple of 8; both pointers device, 16-byte

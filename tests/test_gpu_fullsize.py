@@ -34,7 +34,7 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
 @pytest.mark.parametrize("name,nsel_rows,nq_rows,s_tokens", [("32k", 256, 512, 1024), ("128k", 192, 384, 512)])
-def test_full_size(name, nsel_rows, nq_rows, s_tokens):
+def test_full_size(name, nsel_rows, nq_rows, s_tokens, last_blocks=True):
     from block_sparse_attention_09_b200 import msa
     cfg = CONFIGS[name]
     inp = make_inputs(cfg, seed=11, exact_proxy=True)
@@ -52,6 +52,8 @@ def test_full_size(name, nsel_rows, nq_rows, s_tokens):
 
     # ---- selection of sampled queries, plus every query of the last two blocks
     last = [(b * Hkv + g) * T + i for b in range(cfg.B) for g in range(Hkv) for i in range(T - 256, T)]
+    if not last_blocks:   # the masked-dO check below covers dK/dV; sample the last blocks' rows
+        last = last[::64]
     srows = sample_rows(cfg.B * Hkv * T, nsel_rows, seed=5, must=last)
     idx_o, nsel_o, _ = O.select(m, x["qp"], x["kp"], rows=srows)
     fi, fn = g_idx.reshape(-1, cfg.topk), g_nsel.reshape(-1)
@@ -78,22 +80,22 @@ def test_full_size(name, nsel_rows, nq_rows, s_tokens):
 
     # ---- dK, dV of the last two KV blocks of every group: their selecting
     # queries are all in the last two query blocks, selected above
-    blocks = [(b * Hkv + g) * nb + n for b in range(cfg.B) for g in range(Hkv) for n in (nb - 2, nb - 1)]
-    lrows = [(b * Hq + g * G + hh) * T + i for b in range(cfg.B) for g in range(Hkv)
-             for hh in range(G) for i in range(T - 256, T)]
-    o2, l2 = O.fwd(m, x["q"], x["k"], x["v"], idx_o, nsel_o, rows=lrows)
-    _, D2 = O.bwd_dq(m, x["q"], x["k"], x["v"], x["dout"], o2, l2, idx_o, nsel_o, rows=lrows)
-    dko, dvo = O.bwd_dkdv(m, x["q"], x["k"], x["v"], x["dout"], l2, D2, idx_o, nsel_o, blocks=blocks)
-    sl = slice(T - 256, T)
-    compare("dK last blocks", f32(dk)[:, sl], dko[:, sl])
-    compare("dV last blocks", f32(dv)[:, sl], dvo[:, sl])
+    if last_blocks:
+        blocks = [(b * Hkv + g) * nb + n for b in range(cfg.B) for g in range(Hkv) for n in (nb - 2, nb - 1)]
+        lrows = [(b * Hq + g * G + hh) * T + i for b in range(cfg.B) for g in range(Hkv)
+                 for hh in range(G) for i in range(T - 256, T)]
+        o2, l2 = O.fwd(m, x["q"], x["k"], x["v"], idx_o, nsel_o, rows=lrows)
+        _, D2 = O.bwd_dq(m, x["q"], x["k"], x["v"], x["dout"], o2, l2, idx_o, nsel_o, rows=lrows)
+        dko, dvo = O.bwd_dkdv(m, x["q"], x["k"], x["v"], x["dout"], l2, D2, idx_o, nsel_o, blocks=blocks)
+        sl = slice(T - 256, T)
+        compare("dK last blocks", f32(dk)[:, sl], dko[:, sl])
+        compare("dV last blocks", f32(dv)[:, sl], dvo[:, sl])
 
     # ---- whole-tensor identities (bf16 outputs: each element carries up to
     # 2^-8 relative rounding, so a sum of n of them may be off by about
     # sqrt(n) * 2^-8 * rms; the bound allows five times that)
     gdk = dk.double().cpu().numpy()
     gdv = dv.double().cpu().numpy()
-    dout = x["dout"].astype(np.float64)
     n = T
     for bb in range(cfg.B):
         for g in range(Hkv):
@@ -102,7 +104,7 @@ def test_full_size(name, nsel_rows, nq_rows, s_tokens):
             tol_k = 5 * np.sqrt(n) * 2.0 ** -8 * np.sqrt((kk ** 2).mean()) + 1e-3
             tol_v = 5 * np.sqrt(n) * 2.0 ** -8 * np.sqrt((vv ** 2).mean()) + 1e-3
             assert np.abs(kk.sum(0)).max() <= tol_k, ("sum dK", np.abs(kk.sum(0)).max(), tol_k)
-            want = dout[bb][:, g * G:(g + 1) * G].sum((0, 1))
+            want = x["dout"][bb][:, g * G:(g + 1) * G].sum((0, 1), dtype=np.float64)
             assert np.abs(vv.sum(0) - want).max() <= tol_v, ("sum dV", np.abs(vv.sum(0) - want).max(), tol_v)
 
     # ---- masked dO: heavily shared blocks, fp32 dK/dV, strict bound
