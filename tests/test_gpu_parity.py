@@ -30,14 +30,15 @@ CASES = {
 }
 
 
-def run_and_compare(cfg: Config, inp, report=None, input_scale=1.0):
+def run_and_compare(cfg: Config, inp, report=None, input_scale=1.0, dq_scale=None):
     """input_scale: how much larger than N(0,1) the q/k inputs are; gradient
-    rounding errors grow with it, so the absolute part of the bound does too.
-    dK and dV sum the rounding errors of G heads, which add in quadrature:
-    their absolute bound grows as sqrt(G / 4) beyond the 4 heads per group
-    of the stated workloads."""
+    rounding errors grow with it, so the absolute part of the bound does too
+    (dq_scale, if given, for dQ alone).  dK and dV sum the rounding errors of
+    G heads, which add in quadrature: their absolute bound grows as
+    sqrt(G / 4) beyond the 4 heads per group of the stated workloads."""
     from parity_util import ABS_MAX
     kv_abs = ABS_MAX * input_scale * max(1.0, (cfg.G / 4) ** 0.5)
+    dq_scale = input_scale if dq_scale is None else dq_scale
     dev = to_dev(inp)
     g = gpu_path(dev, cfg.topk, pooled=True)
     x = oracle_inputs(inp)
@@ -56,7 +57,7 @@ def run_and_compare(cfg: Config, inp, report=None, input_scale=1.0):
     dk, dv = O.bwd_dkdv(m, x["q"], x["k"], x["v"], x["dout"], lse, D, idx_o, nsel_o)
     compare("O", f32(g["o"]), o, report=report)
     compare("L", f32(g["lse"]), lse, report=report, rel=0.0)   # fp32 output: plain 2e-2
-    compare("dQ", f32(g["dq"]), dq, report=report, abs_max=ABS_MAX * input_scale)
+    compare("dQ", f32(g["dq"]), dq, report=report, abs_max=ABS_MAX * dq_scale)
     compare("dK", f32(g["dk"]), dk, report=report, abs_max=kv_abs)
     compare("dV", f32(g["dv"]), dv, report=report, abs_max=kv_abs)
     return g
@@ -210,7 +211,11 @@ def test_key_outliers_need_no_fallback():
     from block_sparse_attention_09_b200 import msa
     cfg = Config("outliers", B=1, T=4096, Hq=8, Hkv=2, d=128, dp=64, topk=8, k_outliers=16)
     inp = make_inputs(cfg, seed=3, exact_proxy=True)
-    run_and_compare(cfg, inp, input_scale=8.0)
+    # dQ_i = scale sum_j dS_ij k_j: where an 8x key carries much of a row's
+    # weight, the bf16 rounding of dS (and of O inside D = dO.O) is multiplied
+    # by that key, and dS itself is a difference of two terms of the key's
+    # size -- so dQ's absolute error bound is 8 x 2 times the N(0,1) one.
+    run_and_compare(cfg, inp, input_scale=8.0, dq_scale=16.0)
     dev = to_dev(inp)
     idx, nsel = msa.proxy_select(dev["qp"], dev["kp"], cfg.topk, check=True)
     dims = msa.make_dims(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.d, cfg.dp, cfg.topk)
