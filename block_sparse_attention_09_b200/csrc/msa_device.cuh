@@ -266,6 +266,21 @@ MSA_DEV void tmem_ld32(uint32_t taddr, uint32_t* r)
         : "r"(taddr));
 }
 
+// tcgen05.wait::ld that also names the 32 registers a tcgen05.ld filled: the
+// compiler then cannot move their uses above the wait (used where another
+// load is issued between a load and the use of its registers).
+MSA_DEV void tmem_ld_wait_regs(uint32_t* r)
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 // 32 lanes x 32 bit, 16 consecutive columns per thread.
 MSA_DEV void tmem_st16(uint32_t taddr, const uint32_t* r)
 {
@@ -419,6 +434,23 @@ MSA_DEV float ex2_approx(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA and integer pipes, for x <= 0: range reduction x = n + f
+// (n the nearest integer, |f| <= 1/2), 2^f from a cubic fitted by least
+// squares at Chebyshev nodes on [-1/2, 1/2] (relative error below 8e-5, far
+// under the 2^-9 of the bf16 the weights are stored in), and n added to the
+// exponent field.  2^x below 2^-125 returns 0.  It takes part of the
+// softmax's exponentials off the MUFU pipe, whose rate is a sixteenth of
+// the FMA rate.
+MSA_DEV float ex2_poly(float x)
+{
+    const float xc = fmaxf(x, -125.f);
+    const float r = xc + 12582912.f;           // 1.5 * 2^23: n lands in the low mantissa bits of r
+    const float f = xc - (r - 12582912.f);
+    const float q = fmaf(fmaf(fmaf(0.05508868f, f, 0.24260405f), f, 0.69327623f), f, 0.99992895f);
+    const float y = __int_as_float(__float_as_int(q) + (__float_as_int(r) << 23));
+    return x < -125.f ? 0.f : y;
 }
 
 MSA_DEV uint32_t pack_bf16x2(float lo, float hi)

@@ -203,7 +203,7 @@ proxy_grad_scores_kernel(const __grid_constant__ CUtensorMap tm_kp, ScoreParams 
 // its lanes over the row's selected blocks (up to 4 each), then over the
 // proxy dims for dqp.
 template <int G>
-__global__ void __launch_bounds__(128) proxy_grad_rows_kernel(
+__global__ void __launch_bounds__(128, 4) proxy_grad_rows_kernel(
     const __nv_bfloat16* __restrict__ kp, const int32_t* __restrict__ idx, const int32_t* __restrict__ nsel,
     const int32_t* __restrict__ ptr2, const int32_t* __restrict__ off2, const float* __restrict__ bmass,
     const float* __restrict__ zsel, const int32_t* __restrict__ jsel, int T, int Hp, int dp, int topk, int nblk,
@@ -299,12 +299,12 @@ __global__ void __launch_bounds__(128) proxy_grad_rows_kernel(
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
+            if (32 * k >= ns) continue;   // warp-uniform
+#pragma unroll 8
             for (int l = 0; l < 32; ++l) {
-                const int s = 32 * k + l;
-                if (s >= ns) break;   // warp-uniform
                 const float dzs = __shfl_sync(0xffffffffu, dzk[k], l);
                 const int js = __shfl_sync(0xffffffffu, jk[k], l);
-                if (dzs != 0.f && d0 < dp) {
+                if (32 * k + l < ns && dzs != 0.f && d0 < dp) {
                     const __nv_bfloat162 kv =
                         *reinterpret_cast<const __nv_bfloat162*>(kp + (((int64_t)b * T + js) * Hp + g) * dp + d0);
                     const float2 f = __bfloat1622float2(kv);
@@ -323,43 +323,60 @@ __global__ void __launch_bounds__(128) proxy_grad_rows_kernel(
 }
 
 // dkp of the 256 keys of pair pn of one group, from every entry of the pair
-// list: one CTA, shared-memory fp32 accumulators [256][dp].
+// list: one CTA, shared-memory fp32 accumulators [256][dp + 1] (the odd row
+// stride spreads the rows of different keys over the banks).  Each lane owns
+// one entry at a time: its proxy-query row is loaded whole (all loads in
+// flight together), then added, scaled by dz, into the argmax key's row.
 __global__ void __launch_bounds__(256) proxy_grad_keys_kernel(
     const __nv_bfloat16* __restrict__ qp, const int32_t* __restrict__ ptr2, const int32_t* __restrict__ tok2,
     const int32_t* __restrict__ jsel, const float* __restrict__ dz, int T, int Hp, int dp, int topk, int npair,
     float* __restrict__ dkp)
 {
-    extern __shared__ float acc[];   // [256][dp]
+    extern __shared__ float acc[];   // [256][dp + 1]
+    const int ld = dp + 1;
     const int pn = blockIdx.x, bg = blockIdx.y, b = bg / Hp, g = bg % Hp;
-    for (int x = threadIdx.x; x < 256 * dp; x += blockDim.x) acc[x] = 0.f;
+    for (int x = threadIdx.x; x < 256 * ld; x += blockDim.x) acc[x] = 0.f;
     __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int d0 = 2 * lane;
     const int64_t ebase = (int64_t)bg * T * topk;
     const int e0 = ptr2[(int64_t)bg * (npair + 1) + pn], e1 = ptr2[(int64_t)bg * (npair + 1) + pn + 1];
-    for (int e = e0 + warp; e < e1; e += 8) {
+    const int nvec = dp / 8;   // 16-byte pieces of a proxy row
+    for (int e = e0 + (int)threadIdx.x; e < e1; e += blockDim.x) {
         const int ent = tok2[ebase + e];
         const int i = ent >> 2;
-        float2 q = make_float2(0.f, 0.f);
-        if (d0 < dp)
-            q = __bfloat1622float2(
-                *reinterpret_cast<const __nv_bfloat162*>(qp + (((int64_t)b * T + i) * Hp + g) * dp + d0));
+        float w[2];
+        int key[2];
 #pragma unroll
         for (int sb = 0; sb < 2; ++sb) {
-            if (!((ent >> sb) & 1)) continue;
             const int64_t x = (ebase + e) * 2 + sb;
-            const float w = dz[x];
-            const int key = jsel[x] - 256 * pn;   // 0 .. 255
-            if (d0 < dp && w != 0.f && key >= 0 && key < 256) {
-                atomicAdd(&acc[key * dp + d0], w * q.x);
-                atomicAdd(&acc[key * dp + d0 + 1], w * q.y);
+            const bool on = (ent >> sb) & 1;
+            w[sb] = on ? dz[x] : 0.f;
+            key[sb] = on ? jsel[x] - 256 * pn : -1;   // 0 .. 255
+        }
+        uint4 q[8];
+        const uint4* row = reinterpret_cast<const uint4*>(qp + (((int64_t)b * T + i) * Hp + g) * dp);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) q[c] = c < nvec ? row[c] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int sb = 0; sb < 2; ++sb) {
+            if (w[sb] == 0.f || key[sb] < 0 || key[sb] >= 256) continue;
+            float* dst = acc + key[sb] * ld;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (c >= nvec) break;
+                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q[c]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(h[u]);
+                    atomicAdd(dst + c * 8 + 2 * u, w[sb] * f.x);
+                    atomicAdd(dst + c * 8 + 2 * u + 1, w[sb] * f.y);
+                }
             }
         }
     }
     __syncthreads();
     for (int x = threadIdx.x; x < 256 * dp; x += blockDim.x) {
-        const int key = x / dp, d = x % dp, j = 256 * pn + key;
-        if (j < T) dkp[(((int64_t)b * T + j) * Hp + g) * dp + d] = acc[x];
+        const int k = x / dp, d = x % dp, j = 256 * pn + k;
+        if (j < T) dkp[(((int64_t)b * T + j) * Hp + g) * dp + d] = acc[k * ld + d];
     }
 }
 
@@ -422,7 +439,7 @@ cudaError_t launch_proxy_bwd(const Problem& pr, const CUtensorMap& tm_kp, const 
     }
     if (e != cudaSuccess) return e;
 
-    const size_t kbytes = (size_t)256 * pr.dp * 4;
+    const size_t kbytes = (size_t)256 * (pr.dp + 1) * 4;
     if ((e = cudaFuncSetAttribute(proxy_grad_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kbytes)) !=
         cudaSuccess)
         return e;
