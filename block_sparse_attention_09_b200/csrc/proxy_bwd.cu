@@ -323,10 +323,10 @@ __global__ void __launch_bounds__(128, 4) proxy_grad_rows_kernel(
 }
 
 // dkp of the 256 keys of pair pn of one group, from every entry of the pair
-// list: one CTA, shared-memory fp32 accumulators [256][dp + 1] (the odd row
-// stride spreads the rows of different keys over the banks).  Each lane owns
-// one entry at a time: its proxy-query row is loaded whole (all loads in
-// flight together), then added, scaled by dz, into the argmax key's row.
+// list: one CTA, shared-memory fp32 accumulators [256][dp + 1].  A warp takes
+// four entries at a time, its lanes over the proxy dims (two each): the
+// argmax keys of many rows coincide, so lanes must not add to the same key
+// row at once; the four entries' loads are all in flight together.
 __global__ void __launch_bounds__(256) proxy_grad_keys_kernel(
     const __nv_bfloat16* __restrict__ qp, const int32_t* __restrict__ ptr2, const int32_t* __restrict__ tok2,
     const int32_t* __restrict__ jsel, const float* __restrict__ dz, int T, int Hp, int dp, int topk, int npair,
@@ -337,39 +337,40 @@ __global__ void __launch_bounds__(256) proxy_grad_keys_kernel(
     const int pn = blockIdx.x, bg = blockIdx.y, b = bg / Hp, g = bg % Hp;
     for (int x = threadIdx.x; x < 256 * ld; x += blockDim.x) acc[x] = 0.f;
     __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int d0 = 2 * lane;
     const int64_t ebase = (int64_t)bg * T * topk;
     const int e0 = ptr2[(int64_t)bg * (npair + 1) + pn], e1 = ptr2[(int64_t)bg * (npair + 1) + pn + 1];
-    const int nvec = dp / 8;   // 16-byte pieces of a proxy row
-    for (int e = e0 + (int)threadIdx.x; e < e1; e += blockDim.x) {
-        const int ent = tok2[ebase + e];
-        const int i = ent >> 2;
-        float w[2];
-        int key[2];
-#pragma unroll
-        for (int sb = 0; sb < 2; ++sb) {
-            const int64_t x = (ebase + e) * 2 + sb;
-            const bool on = (ent >> sb) & 1;
-            w[sb] = on ? dz[x] : 0.f;
-            key[sb] = on ? jsel[x] - 256 * pn : -1;   // 0 .. 255
+    constexpr int kE = 4;   // entries per warp step
+    for (int base = e0 + warp * kE; base < e1; base += 8 * kE) {
+        // lane l < 2 kE loads (entry l / 2, block l % 2): its flags, weight and key
+        const int le = base + (lane >> 1), lsb = lane & 1;
+        int lent = 0, lkey = -1;
+        float lw = 0.f;
+        if (lane < 2 * kE && le < e1) {
+            lent = tok2[ebase + le];
+            if ((lent >> lsb) & 1) {
+                const int64_t x = (ebase + le) * 2 + lsb;
+                lw = dz[x];
+                lkey = jsel[x] - 256 * pn;   // 0 .. 255
+            }
         }
-        uint4 q[8];
-        const uint4* row = reinterpret_cast<const uint4*>(qp + (((int64_t)b * T + i) * Hp + g) * dp);
+        float2 q[kE];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) q[c] = c < nvec ? row[c] : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < kE; ++u) {
+            const int ent = __shfl_sync(0xffffffffu, lent, 2 * u);
+            q[u] = make_float2(0.f, 0.f);
+            if (base + u < e1 && d0 < dp)
+                q[u] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+                    qp + (((int64_t)b * T + (ent >> 2)) * Hp + g) * dp + d0));
+        }
 #pragma unroll
-        for (int sb = 0; sb < 2; ++sb) {
-            if (w[sb] == 0.f || key[sb] < 0 || key[sb] >= 256) continue;
-            float* dst = acc + key[sb] * ld;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                if (c >= nvec) break;
-                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q[c]);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 f = __bfloat1622float2(h[u]);
-                    atomicAdd(dst + c * 8 + 2 * u, w[sb] * f.x);
-                    atomicAdd(dst + c * 8 + 2 * u + 1, w[sb] * f.y);
-                }
+        for (int u = 0; u < 2 * kE; ++u) {
+            const float w = __shfl_sync(0xffffffffu, lw, u);
+            const int key = __shfl_sync(0xffffffffu, lkey, u);
+            if (w != 0.f && key >= 0 && key < 256 && d0 < dp) {
+                atomicAdd(acc + key * ld + d0, w * q[u >> 1].x);
+                atomicAdd(acc + key * ld + d0 + 1, w * q[u >> 1].y);
             }
         }
     }

@@ -366,19 +366,22 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
         // cut at the query (causal)
         auto block_max = [&](uint32_t ta, bool diag) -> float {
             float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+            // four quarters of 32 columns, the next quarter's load in flight
+            // while one is reduced
+            uint32_t va[32], vb[32];
+            tmem_ld32(ta, va);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t v[64];
-                tmem_ld32(ta + h * 64, v);
-                tmem_ld32(ta + h * 64 + 32, v + 32);
-                tmem_ld_wait();
+            for (int qd = 0; qd < 4; ++qd) {
+                uint32_t* v = (qd & 1) ? vb : va;
+                tmem_ld_wait_regs(v);
+                if (qd + 1 < 4) tmem_ld32(ta + (qd + 1) * 32, (qd & 1) ? va : vb);
                 if (diag) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (h * 64 + c > r) v[c] = __float_as_uint(-INFINITY);
+                    for (int c = 0; c < 32; ++c)
+                        if (qd * 32 + c > r) v[c] = __float_as_uint(-INFINITY);
                 }
 #pragma unroll
-                for (int c = 0; c < 64; c += 8) {
+                for (int c = 0; c < 32; c += 8) {
                     m0 = fmax3(m0, __uint_as_float(v[c + 0]), __uint_as_float(v[c + 1]));
                     m1 = fmax3(m1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
                     m2 = fmax3(m2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));

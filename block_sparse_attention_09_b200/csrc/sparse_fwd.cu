@@ -280,44 +280,21 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tc_fence_after();
                 // last key of block n0 + s this row reads (-1: none)
                 const int cmax = !((flags >> s) & 1) ? -1 : (((i >> 7) == n0 + s) ? (i & 127) : 127);
-                // a block the row did not select gets the shift +inf: every weight
-                // becomes exp2(-inf) = 0 with no compare; only a warp holding a
-                // diagonal row (keys after the query) takes the masked path
-                const float mhs = cmax < 0 ? INFINITY : mh;
-                const bool plain = __all_sync(0xffffffffu, cmax < 0 || cmax == 127);
                 const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)s * 128u);
-                // pieces of 32 columns, the next one's load in flight while this one is computed
-                uint32_t va[32], vb[32];
-                tmem_ld32(ta, va);
 #pragma unroll
                 for (int piece = 0; piece < 4; ++piece) {
-                    uint32_t* v = (piece & 1) ? vb : va;
-                    uint32_t pk[16];
-                    tmem_ld_wait_regs(v);
-                    if (piece + 1 < 4) tmem_ld32(ta + (piece + 1) * 32, (piece & 1) ? va : vb);
-                    if (plain) {
+                    uint32_t v[32], pk[16];
+                    tmem_ld32(ta + piece * 32, v);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float x0 = fmaf(__uint_as_float(v[2 * e]), p.c1, -mhs);
-                            const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mhs);
-                            // one pair in four on the FMA pipe, the rest on MUFU
-                            const float p0 = (e & 3) == 3 ? ex2_poly(x0) : ex2_approx(x0);
-                            const float p1 = (e & 3) == 3 ? ex2_poly(x1) : ex2_approx(x1);
-                            pk[e] = pack_bf16x2(p0, p1);
-                            // normalise by the weights the PV product actually uses (bf16), so
-                            // that O is an exact convex combination of the selected values
-                            ls += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int c0 = piece * 32 + 2 * e;
-                            const float p0 = c0 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e]), p.c1, -mh)) : 0.f;
-                            const float p1 =
-                                c0 + 1 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mh)) : 0.f;
-                            pk[e] = pack_bf16x2(p0, p1);
-                            ls += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
-                        }
+                    for (int e = 0; e < 16; ++e) {
+                        const int c0 = piece * 32 + 2 * e;
+                        const float p0 = c0 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e]), p.c1, -mh)) : 0.f;
+                        const float p1 = c0 + 1 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mh)) : 0.f;
+                        pk[e] = pack_bf16x2(p0, p1);
+                        // normalise by the weights the PV product actually uses (bf16), so
+                        // that O is an exact convex combination of the selected values
+                        ls += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
                     }
                     tmem_st16(ta + piece * 16, pk);   // P overwrites S columns already read
                 }
