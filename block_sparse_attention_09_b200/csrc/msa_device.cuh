@@ -436,23 +436,6 @@ MSA_DEV float ex2_approx(float x)
     return y;
 }
 
-// 2^x on the FMA and integer pipes, for x <= 0: range reduction x = n + f
-// (n the nearest integer, |f| <= 1/2), 2^f from a cubic fitted by least
-// squares at Chebyshev nodes on [-1/2, 1/2] (relative error below 8e-5, far
-// under the 2^-9 of the bf16 the weights are stored in), and n added to the
-// exponent field.  2^x below 2^-125 returns 0.  It takes part of the
-// softmax's exponentials off the MUFU pipe, whose rate is a sixteenth of
-// the FMA rate.
-MSA_DEV float ex2_poly(float x)
-{
-    const float xc = fmaxf(x, -125.f);
-    const float r = xc + 12582912.f;           // 1.5 * 2^23: n lands in the low mantissa bits of r
-    const float f = xc - (r - 12582912.f);
-    const float q = fmaf(fmaf(fmaf(0.05508868f, f, 0.24260405f), f, 0.69327623f), f, 0.99992895f);
-    const float y = __int_as_float(__float_as_int(q) + (__float_as_int(r) << 23));
-    return x < -125.f ? 0.f : y;
-}
-
 MSA_DEV uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

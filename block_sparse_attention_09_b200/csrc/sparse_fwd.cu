@@ -44,7 +44,8 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 448;   // w0 TMA(K,V) | w1 MMA | w2-5 gather | w6-9 softmax | w10-13 O out
+constexpr int kThreads = 512;   // w0 TMA(K,V) | w1 MMA | w2-3 gather | w4-7 softmax of block 2p | w8-11 O out | w12-15 softmax of block 2p+1
+constexpr int kGather = 64;     // gather threads
 constexpr int kQStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSumLow = 7.703719777548943e-34f;     // 2^-110: row sums outside [kSumLow, kSumHigh]
@@ -137,7 +138,7 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        for (int s = 0; s < kQStages; ++s) { mbar_init(&q_full[s], 128); mbar_init(&q_empty[s], 1); }
+        for (int s = 0; s < kQStages; ++s) { mbar_init(&q_full[s], kGather); mbar_init(&q_empty[s], 1); }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], 128);
@@ -221,8 +222,8 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             umma_commit(fin);
             mbar_drain(fin, 0);
         }
-    } else if (warp < 6) {
-        // ---------------- query gather (cp.async, 128 threads) ----------------
+    } else if (warp < 4) {
+        // ---------------- query gather (cp.async, 64 threads) ----------------
         const int tid = threadIdx.x - 64;
         constexpr int kPieces = 128 * D / 8;           // 16-byte pieces per chunk
         constexpr int kRowPieces = D / 8;
@@ -232,8 +233,8 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (use > 0 && !mbar_wait(&q_empty[s], (use - 1) & 1u, wc, code0 + 4)) break;
             const uint32_t qs = smem_u32(q_st + s * kTile);
 #pragma unroll 4
-            for (int it = 0; it < kPieces / 128; ++it) {
-                const int piece = it * 128 + tid;
+            for (int it = 0; it < kPieces / kGather; ++it) {
+                const int piece = it * kGather + tid;
                 const int row = piece / kRowPieces, ch = piece % kRowPieces;
                 const int t = row & (p.tpc - 1), hh = row >> (7 - p.lgG);
                 const int jj = c * p.tpc + t;
@@ -249,8 +250,10 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_arrive(&q_full[s]);
         }
         cp_async_wait<0>();
-    } else if (warp < 10) {
+    } else if (warp < 8 || warp >= 12) {
         // ---------------- softmax: P = exp2(S*c1 - m_i) ----------------
+        // warps 4-7 take block 2p, warps 12-15 block 2p+1: the two blocks of a
+        // chunk are exponentiated at the same time on different warps
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32);
         const int t = r & (p.tpc - 1), hh = r >> (7 - p.lgG), h = g * G + hh;
@@ -273,28 +276,52 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             float l = 0.f;
             bool ok = true;
             const int64_t ent_idx = (int64_t)bg * p.T * p.topk + item.beg + c * p.tpc + t;   // this row's entry
-            for (int s = 0; s < nsub; ++s) {
+            const int s_first = warp < 8 ? 0 : 1;
+            if (s_first >= nsub) break;   // no second block in this item: nothing for this group
+            for (int s = s_first; s < s_first + 1; ++s) {
                 float ls = 0.f;
                 ok = mbar_wait(&s_full[s], (uint32_t)c & 1u, wc, code0 + 5);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
                 // last key of block n0 + s this row reads (-1: none)
                 const int cmax = !((flags >> s) & 1) ? -1 : (((i >> 7) == n0 + s) ? (i & 127) : 127);
+                // a block the row did not select gets the shift +inf: every weight
+                // becomes exp2(-inf) = 0 with no compare; only a warp holding a
+                // diagonal row (keys after the query) takes the masked path
+                const float mhs = cmax < 0 ? INFINITY : mh;
+                const bool plain = __all_sync(0xffffffffu, cmax < 0 || cmax == 127);
                 const uint32_t ta = tmem_addr(tmem, lane_base, (uint32_t)s * 128u);
+                // pieces of 32 columns, the next one's load in flight while this one is computed
+                uint32_t va[32], vb[32];
+                tmem_ld32(ta, va);
 #pragma unroll
                 for (int piece = 0; piece < 4; ++piece) {
-                    uint32_t v[32], pk[16];
-                    tmem_ld32(ta + piece * 32, v);
-                    tmem_ld_wait();
+                    uint32_t* v = (piece & 1) ? vb : va;
+                    uint32_t pk[16];
+                    tmem_ld_wait_regs(v);
+                    if (piece + 1 < 4) tmem_ld32(ta + (piece + 1) * 32, (piece & 1) ? va : vb);
+                    if (plain) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c0 = piece * 32 + 2 * e;
-                        const float p0 = c0 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e]), p.c1, -mh)) : 0.f;
-                        const float p1 = c0 + 1 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mh)) : 0.f;
-                        pk[e] = pack_bf16x2(p0, p1);
-                        // normalise by the weights the PV product actually uses (bf16), so
-                        // that O is an exact convex combination of the selected values
-                        ls += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+                        for (int e = 0; e < 16; ++e) {
+                            const float x0 = fmaf(__uint_as_float(v[2 * e]), p.c1, -mhs);
+                            const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mhs);
+                            const float p0 = ex2_approx(x0);
+                            const float p1 = ex2_approx(x1);
+                            pk[e] = pack_bf16x2(p0, p1);
+                            // normalise by the weights the PV product actually uses (bf16), so
+                            // that O is an exact convex combination of the selected values
+                            ls += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int c0 = piece * 32 + 2 * e;
+                            const float p0 = c0 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e]), p.c1, -mh)) : 0.f;
+                            const float p1 =
+                                c0 + 1 <= cmax ? ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), p.c1, -mh)) : 0.f;
+                            pk[e] = pack_bf16x2(p0, p1);
+                            ls += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+                        }
                     }
                     tmem_st16(ta + piece * 16, pk);   // P overwrites S columns already read
                 }
@@ -320,7 +347,7 @@ fwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int t = r & (p.tpc - 1), hh = r >> (7 - p.lgG);
         const int half_tok = p.tpc >> 1;                       // tokens per half
         const int my_half = t >= half_tok ? 1 : 0;
-        const int tid = threadIdx.x - 320;                     // token (within a half) this thread reduces
+        const int tid = threadIdx.x - 256;                     // token (within a half) this thread reduces
         const uint32_t stg = smem_u32(o_stg);
         const uint32_t my_row = stg + (uint32_t)(t - my_half * half_tok) * tok_stride + (uint32_t)hh * D * 4u;
         auto tok_at = [&](int cc, int hf) {
