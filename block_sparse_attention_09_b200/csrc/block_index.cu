@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(1024) index_ptr_kernel(const int32_t* __restri
 // list (ptr[n] + off[qb][n] onward), in ascending order: a warp writes it
 // from the tile's membership mask, lane l taking bit l of each 32-bit word, so
 // the stores of one word land on consecutive positions.
-__global__ void __launch_bounds__(128) index_fill_kernel(const int32_t* __restrict__ idx,
+__global__ void __launch_bounds__(512) index_fill_kernel(const int32_t* __restrict__ idx,
                                                          const int32_t* __restrict__ nsel, int T, int topk,
                                                          int nblk, int npair, int qb0, const int32_t* __restrict__ off,
                                                          const int32_t* __restrict__ ptr, int32_t* __restrict__ tok,
@@ -141,20 +141,30 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t* __restri
     const int qb = qb0 + (int)blockIdx.x, bg = blockIdx.y;
     build_masks(mask, idx, nsel, T, topk, qb, bg);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (int)(blockDim.x >> 5);
     const uint32_t below = (1u << lane) - 1u;
+    // A warp takes 32 consecutive blocks at a time: their list offsets are
+    // loaded together (lane j: block n0 + j, one coalesced load each), so the
+    // per-block loop below runs on shared memory and shuffles only.
     {
         const int32_t* offrow = off + ((int64_t)bg * nblk + qb) * nblk;
         const int32_t* p = ptr + (int64_t)bg * (nblk + 1);
         int32_t* out = tok + (int64_t)bg * T * topk;
-        for (int n = warp; n <= qb; n += 4) {
-            const uint32_t m0 = mask[n * 4], m1 = mask[n * 4 + 1], m2 = mask[n * 4 + 2], m3 = mask[n * 4 + 3];
-            if ((m0 | m1 | m2 | m3) == 0u) continue;
-            int pos = p[n] + offrow[n];
-            const uint32_t mw[4] = {m0, m1, m2, m3};
+        for (int n0 = warp * 32; n0 <= qb; n0 += nwarps * 32) {
+            const int nl = n0 + lane;
+            const int base = nl <= qb ? p[nl] + offrow[nl] : 0;
+            const int nn = min(32, qb + 1 - n0);
+            for (int j = 0; j < nn; ++j) {
+                const int n = n0 + j;
+                const uint32_t m0 = mask[n * 4], m1 = mask[n * 4 + 1], m2 = mask[n * 4 + 2], m3 = mask[n * 4 + 3];
+                int pos = __shfl_sync(0xffffffffu, base, j);
+                if ((m0 | m1 | m2 | m3) == 0u) continue;
+                const uint32_t mw[4] = {m0, m1, m2, m3};
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                if ((mw[w] >> lane) & 1u) out[pos + __popc(mw[w] & below)] = qb * 128 + w * 32 + lane;
-                pos += __popc(mw[w]);
+                for (int w = 0; w < 4; ++w) {
+                    if ((mw[w] >> lane) & 1u) out[pos + __popc(mw[w] & below)] = qb * 128 + w * 32 + lane;
+                    pos += __popc(mw[w]);
+                }
             }
         }
     }
@@ -162,23 +172,29 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t* __restri
     const int32_t* offrow = off2 + ((int64_t)bg * nblk + qb) * npair;
     const int32_t* p = ptr2 + (int64_t)bg * (npair + 1);
     int32_t* out = tok2 + (int64_t)bg * T * topk;
-    for (int pp = warp; 2 * pp <= qb; pp += 4) {
-        uint32_t a[4], c[4], u = 0u;
+    for (int p0 = warp * 32; 2 * p0 <= qb; p0 += nwarps * 32) {
+        const int pl = p0 + lane;
+        const int base = 2 * pl <= qb ? p[pl] + offrow[pl] : 0;
+        const int nn = min(32, qb / 2 + 1 - p0);
+        for (int j = 0; j < nn; ++j) {
+            const int pp = p0 + j;
+            uint32_t a[4], c[4], u = 0u;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            a[w] = mask[(2 * pp) * 4 + w];
-            c[w] = 2 * pp + 1 <= qb ? mask[(2 * pp + 1) * 4 + w] : 0u;
-            u |= a[w] | c[w];
-        }
-        if (u == 0u) continue;
-        int pos = p[pp] + offrow[pp];
+            for (int w = 0; w < 4; ++w) {
+                a[w] = mask[(2 * pp) * 4 + w];
+                c[w] = 2 * pp + 1 <= qb ? mask[(2 * pp + 1) * 4 + w] : 0u;
+                u |= a[w] | c[w];
+            }
+            int pos = __shfl_sync(0xffffffffu, base, j);
+            if (u == 0u) continue;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const uint32_t mw = a[w] | c[w];
-            if ((mw >> lane) & 1u)
-                out[pos + __popc(mw & below)] =
-                    ((qb * 128 + w * 32 + lane) << 2) | (int)((a[w] >> lane) & 1u) | (int)(((c[w] >> lane) & 1u) << 1);
-            pos += __popc(mw);
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t mw = a[w] | c[w];
+                if ((mw >> lane) & 1u)
+                    out[pos + __popc(mw & below)] = ((qb * 128 + w * 32 + lane) << 2) | (int)((a[w] >> lane) & 1u) |
+                                                    (int)(((c[w] >> lane) & 1u) << 1);
+                pos += __popc(mw);
+            }
         }
     }
 }
@@ -219,7 +235,7 @@ cudaError_t launch_block_index(const Problem& pr, const int32_t* idx, const int3
     count_launches(1);
     index_ptr_kernel<<<dim3(BH, 2), 1024, 0, st>>>(tot, ptr, tot2, ptr2, pr.nblk, npair);
     count_launches(1);
-    index_fill_kernel<<<g1, 128, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, npair, pr.qb0, cnt, ptr, tok,
+    index_fill_kernel<<<g1, 512, mask_bytes, st>>>(idx, nsel, pr.T, pr.topk, pr.nblk, npair, pr.qb0, cnt, ptr, tok,
                                                    cnt2, ptr2, tok2);
     count_launches(1);
     return cudaGetLastError();

@@ -47,7 +47,7 @@ namespace {
 constexpr int kThreads = 448;             // warp 0: TMA, 1: MMA, 2-9: pooling, 10-13: selection
 constexpr uint32_t kTileBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle slab)
 constexpr int kPend = 10;                  // pending slots per row (merge once one row holds 8)
-constexpr int kRing = 4;                   // pairs of block maxima in flight from pooling to selection
+constexpr int kRing = 8;                   // pairs of block maxima in flight from pooling to selection
 
 struct Params {
     int B, T, Hp, dp, nblk, topk;
@@ -444,18 +444,27 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
                 ++npend;
             }
         };
-        for (int k = 0; k < npairs; ++k) {
+        // two pairs per handshake: both slots' maxima are read together
+        for (int k = 0; k < npairs; k += 2) {
+            const bool two = k + 1 < npairs;
             const int hi = ntiles - 1 - 2 * k, lo = hi - 1;
-            const int slot = k % kRing;
-            const bool ok = mbar_wait(&pm_full[slot], (uint32_t)(k / kRing) & 1u, wc, code0 + 6);
+            const int slot = k % kRing, slot1 = (k + 1) % kRing;
+            bool ok = mbar_wait(&pm_full[slot], (uint32_t)(k / kRing) & 1u, wc, code0 + 6);
+            if (ok && two) ok = mbar_wait(&pm_full[slot1], (uint32_t)((k + 1) / kRing) & 1u, wc, code0 + 6);
             if (!__all_sync(0xffffffffu, ok)) break;
             const float mhi = pm[(slot * 2 + 1) * 128 + r], mlo = pm[slot * 2 * 128 + r];
+            const float mhi1 = two ? pm[(slot1 * 2 + 1) * 128 + r] : 0.f, mlo1 = two ? pm[slot1 * 2 * 128 + r] : 0.f;
             mbar_arrive(&pm_empty[slot]);
+            if (two) mbar_arrive(&pm_empty[slot1]);
             consume(hi, mhi);
             if (lo >= 0) consume(lo, mlo);
-            // one vote per pair: at most two appends per pair, so a list
-            // holding 8 still has room for the next pair
-            if (need_heap && cnt == k1 && __any_sync(0xffffffffu, npend >= kPend - 2)) merge_pending();
+            if (two) {
+                consume(hi - 2, mhi1);
+                if (lo - 2 >= 0) consume(lo - 2, mlo1);
+            }
+            // one vote per two pairs: at most four appends, so a list holding
+            // 6 still has room for the next two pairs
+            if (need_heap && cnt == k1 && __any_sync(0xffffffffu, npend >= kPend - 4)) merge_pending();
         }
         if (need_heap && cnt == k1) merge_pending();
         const bool go = __all_sync(0xffffffffu, !*abort_flag);
