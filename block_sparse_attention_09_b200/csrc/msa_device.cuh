@@ -411,6 +411,28 @@ __device__ __forceinline__ bool build_masks(uint32_t* mask, const int32_t* idx, 
 }
 
 // Active query row r (0 .. B*(T-q0)*Hq - 1: the rows q0 .. T-1 of every batch
+// and head, head fastest) -> (b, i, h).  Small: r < 2^31, so 32-bit division
+// suffices (the 64-bit one costs several times as many instructions).
+template <bool Small>
+MSA_DEV void active_coords(int64_t r, int T, int Hq, int q0, int& b, int& i, int& h)
+{
+    const int Tq = T - q0;
+    if (Small) {
+        const uint32_t ru = (uint32_t)r, hq = (uint32_t)Hq, tq = (uint32_t)Tq;
+        const uint32_t bi = ru / hq;
+        h = (int)(ru - bi * hq);
+        const uint32_t bb = bi / tq;
+        i = q0 + (int)(bi - bb * tq);
+        b = (int)bb;
+    } else {
+        h = (int)(r % Hq);
+        const int64_t bi = r / Hq;
+        i = q0 + (int)(bi % Tq);
+        b = (int)(bi / Tq);
+    }
+}
+
+// Active query row r (0 .. B*(T-q0)*Hq - 1: the rows q0 .. T-1 of every batch
 // and head) -> its flat index (b*T + i)*Hq + h in a [B][T][Hq] tensor.
 MSA_DEV int64_t active_row(int64_t r, int T, int Hq, int q0)
 {

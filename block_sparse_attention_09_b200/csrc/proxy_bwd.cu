@@ -322,11 +322,17 @@ __global__ void __launch_bounds__(128, 4) proxy_grad_rows_kernel(
     }
 }
 
-// dkp of the 256 keys of pair pn of one group, from every entry of the pair
-// list: one CTA, shared-memory fp32 accumulators [256][dp + 1].  A warp takes
+// dkp of the 256 keys of pair pn of one group, from the entries of the pair
+// list: up to kKeySplit CTAs per pair, each over its share of the entries
+// with shared-memory fp32 accumulators [256][dp + 1], added into dkp at the
+// end (the pair holding block 0 is selected by every row: at 1M tokens one
+// CTA would walk a million entries).  A warp takes
 // four entries at a time, its lanes over the proxy dims (two each): the
 // argmax keys of many rows coincide, so lanes must not add to the same key
 // row at once; the four entries' loads are all in flight together.
+constexpr int kKeyMinChunk = 2048;   // entries: fewer go to one CTA
+constexpr int kKeySplit = 16;        // at most this many CTAs per pair
+
 __global__ void __launch_bounds__(256) proxy_grad_keys_kernel(
     const __nv_bfloat16* __restrict__ qp, const int32_t* __restrict__ ptr2, const int32_t* __restrict__ tok2,
     const int32_t* __restrict__ jsel, const float* __restrict__ dz, int T, int Hp, int dp, int topk, int npair,
@@ -335,12 +341,19 @@ __global__ void __launch_bounds__(256) proxy_grad_keys_kernel(
     extern __shared__ float acc[];   // [256][dp + 1]
     const int ld = dp + 1;
     const int pn = blockIdx.x, bg = blockIdx.y, b = bg / Hp, g = bg % Hp;
+    // this CTA's share of the pair's entry list: gridDim.z equal parts of at
+    // least kKeyMinChunk entries (a heavily shared pair, such as the one
+    // holding block 0, is spread over several CTAs instead of one)
+    const int p0 = ptr2[(int64_t)bg * (npair + 1) + pn], p1 = ptr2[(int64_t)bg * (npair + 1) + pn + 1];
+    const int cs = max(kKeyMinChunk, (p1 - p0 + (int)gridDim.z - 1) / (int)gridDim.z);
+    const int e0 = p0 + (int)blockIdx.z * cs;
+    if (e0 >= p1) return;   // CTA-uniform
+    const int e1 = min(p1, e0 + cs);
     for (int x = threadIdx.x; x < 256 * ld; x += blockDim.x) acc[x] = 0.f;
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int d0 = 2 * lane;
     const int64_t ebase = (int64_t)bg * T * topk;
-    const int e0 = ptr2[(int64_t)bg * (npair + 1) + pn], e1 = ptr2[(int64_t)bg * (npair + 1) + pn + 1];
     constexpr int kE = 4;   // entries per warp step
     for (int base = e0 + warp * kE; base < e1; base += 8 * kE) {
         // lane l < 2 kE loads (entry l / 2, block l % 2): its flags, weight and key
@@ -375,9 +388,12 @@ __global__ void __launch_bounds__(256) proxy_grad_keys_kernel(
         }
     }
     __syncthreads();
+    // add the partial sums into dkp (zeroed before the launch); most keys of
+    // a pair are nobody's argmax and are skipped
     for (int x = threadIdx.x; x < 256 * dp; x += blockDim.x) {
         const int k = x / dp, d = x % dp, j = 256 * pn + k;
-        if (j < T) dkp[(((int64_t)b * T + j) * Hp + g) * dp + d] = acc[k * ld + d];
+        const float v = acc[k * ld + d];
+        if (j < T && v != 0.f) atomicAdd(dkp + (((int64_t)b * T + j) * Hp + g) * dp + d, v);
     }
 }
 
@@ -444,7 +460,9 @@ cudaError_t launch_proxy_bwd(const Problem& pr, const CUtensorMap& tm_kp, const 
     if ((e = cudaFuncSetAttribute(proxy_grad_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kbytes)) !=
         cudaSuccess)
         return e;
-    proxy_grad_keys_kernel<<<dim3((unsigned)npair, (unsigned)(pr.B * pr.Hp)), 256, kbytes, st>>>(
+    if ((e = cudaMemsetAsync(dkp, 0, sizeof(float) * (size_t)pr.B * pr.T * pr.Hp * pr.dp, st)) != cudaSuccess)
+        return e;
+    proxy_grad_keys_kernel<<<dim3((unsigned)npair, (unsigned)(pr.B * pr.Hp), (unsigned)kKeySplit), 256, kbytes, st>>>(
         (const __nv_bfloat16*)qp, ptr2, tok2, jsel, dz, pr.T, pr.Hp, pr.dp, pr.topk, npair, dkp);
     count_launches(1);
     return cudaGetLastError();

@@ -478,7 +478,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 // D_i = dO_i . O_i per computed query row (rows q0 .. T-1; bf16 inputs, fp32
 // sum); D/8 lanes per row.
-template <int D>
+template <int D, bool Small>
 __global__ void __launch_bounds__(256) bwd_dsum_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout, int B, int T,
                                                        int Hq, int q0, float* __restrict__ dsum)
@@ -488,7 +488,9 @@ __global__ void __launch_bounds__(256) bwd_dsum_kernel(const __nv_bfloat16* __re
     const int64_t ar = gt / LPR;
     const int sub = (int)(gt % LPR);
     const bool ok = ar < (int64_t)B * (T - q0) * Hq;
-    const int64_t row = ok ? active_row(ar, T, Hq, q0) : 0;
+    int b = 0, i = 0, h = 0;
+    if (ok) active_coords<Small>(ar, T, Hq, q0, b, i, h);
+    const int64_t row = ((int64_t)b * T + i) * Hq + h;
     float s = 0.f;
     if (ok) {
         const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + sub * 8);
@@ -504,12 +506,7 @@ __global__ void __launch_bounds__(256) bwd_dsum_kernel(const __nv_bfloat16* __re
     }
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (ok && sub == 0) {
-        const int h = (int)(row % Hq);
-        const int64_t bi = row / Hq;
-        const int i = (int)(bi % T), b = (int)(bi / T);
-        dsum[((int64_t)b * Hq + h) * T + i] = s;
-    }
+    if (ok && sub == 0) dsum[((int64_t)b * Hq + h) * T + i] = s;
 }
 
 // fp32 accumulator -> bf16, 8 elements per thread.
@@ -567,8 +564,12 @@ cudaError_t launch_bwd_d(const Problem& pr, const void* q, const void* dout, con
     if ((e = cudaMemsetAsync(dkacc, 0, sizeof(float) * kv_elems, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dvacc, 0, sizeof(float) * kv_elems, st)) != cudaSuccess) return e;
     const int64_t th = pr.rows_q_active() * (D / 8);
-    bwd_dsum_kernel<D><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(
-        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, pr.q0, dsum);
+    if (th < ((int64_t)1 << 31))
+        bwd_dsum_kernel<D, true><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(
+            (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, pr.q0, dsum);
+    else
+        bwd_dsum_kernel<D, false><<<(unsigned)((th + 255) / 256), 256, 0, st>>>(
+            (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, pr.B, pr.T, pr.Hq, pr.q0, dsum);
     count_launches(1);
 
     BwdParams p;

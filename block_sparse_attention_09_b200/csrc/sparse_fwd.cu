@@ -38,6 +38,8 @@
 // two-pass softmax.
 #include <math.h>
 
+#include <type_traits>
+
 #include "msa_device.cuh"
 #include "msa_internal.h"
 
@@ -485,37 +487,64 @@ __global__ void __launch_bounds__(256) fwd_shift_kernel(const __nv_bfloat16* __r
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, off));
+    // D/32 consecutive elements per lane: one 4- or 8-byte load per row
+    using Vec = typename std::conditional<EPL == 4, uint2, uint32_t>::type;
+    auto unpack = [](Vec v, float* f) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int e = 0; e < EPL / 2; ++e) {
+            const float2 x = __bfloat1622float2(h2[e]);
+            f[2 * e] = x.x;
+            f[2 * e + 1] = x.y;
+        }
+    };
     float kv[EPL];
-    {
-        const __nv_bfloat16* kr = k + (((int64_t)b * T + i) * Hkv + g) * D + lane * EPL;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) kv[e] = __bfloat162float(kr[e]);
-    }
+    unpack(*reinterpret_cast<const Vec*>(k + (((int64_t)b * T + i) * Hkv + g) * D + lane * EPL), kv);
     const float c1abs = fabsf(c1);
-    for (int hh = 0; hh < G; ++hh) {
-        const int h = g * G + hh;
-        const __nv_bfloat16* qr = q + (((int64_t)b * T + i) * Hq + h) * D + lane * EPL;
-        float ss = 0.f, dot = 0.f;
+    // the group's G query rows are consecutive: four heads' loads in flight at a time
+    const __nv_bfloat16* qg = q + (((int64_t)b * T + i) * Hq + g * G) * D + lane * EPL;
+    for (int h0 = 0; h0 < G; h0 += 4) {
+        const int nh = min(4, G - h0);
+        Vec qv[4];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-            const float x = __bfloat162float(qr[e]);
-            ss = fmaf(x, x, ss);
-            dot = fmaf(x, kv[e], dot);
+        for (int u = 0; u < 4; ++u)
+            if (u < nh) qv[u] = *reinterpret_cast<const Vec*>(qg + (int64_t)(h0 + u) * D);
+        float ss[4], dot[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float x[EPL];
+            unpack(u < nh ? qv[u] : Vec{}, x);
+            ss[u] = 0.f;
+            dot[u] = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+                ss[u] = fmaf(x[e], x[e], ss[u]);
+                dot[u] = fmaf(x[e], kv[e], dot[u]);
+            }
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
-            ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            dot += __shfl_xor_sync(0xffffffffu, dot, off);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
+                dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], off);
+            }
         }
-        if (lane == 0)
-            shift[((int64_t)b * Hq + h) * T + i] = fminf(c1abs * sqrtf(ss) * km, c1 * dot + kShiftSlack);
+        if (lane < nh) {
+            float su = ss[0], du = dot[0];
+#pragma unroll
+            for (int u = 1; u < 4; ++u)
+                if (lane == u) { su = ss[u]; du = dot[u]; }
+            const int h = g * G + h0 + lane;
+            shift[((int64_t)b * Hq + h) * T + i] = fminf(c1abs * sqrtf(su) * km, c1 * du + kShiftSlack);
+        }
     }
 }
 
 // O = O_acc / l (bf16), L = (m + log2 l) ln 2 for the computed rows (q0 ..
 // T-1); rows whose l is outside [kSumLow, kSumHigh] or not finite are listed
 // (count in status word 2).
-template <int D>
+template <int D, bool Small>
 __global__ void __launch_bounds__(256) fwd_finalize_kernel(const float* __restrict__ oacc,
                                                            const float* __restrict__ lacc,
                                                            const float* __restrict__ shift, int B, int T,
@@ -528,10 +557,9 @@ __global__ void __launch_bounds__(256) fwd_finalize_kernel(const float* __restri
     const int64_t ar = gt / LPR;
     const int sub = (int)(gt % LPR);
     if (ar >= (int64_t)B * (T - q0) * Hq) return;
-    const int64_t row = active_row(ar, T, Hq, q0);   // (b*T + i)*Hq + h
-    const int h = (int)(row % Hq);
-    const int64_t bi = row / Hq;
-    const int i = (int)(bi % T), b = (int)(bi / T);
+    int b, i, h;
+    active_coords<Small>(ar, T, Hq, q0, b, i, h);
+    const int64_t row = ((int64_t)b * T + i) * Hq + h;
     const int64_t lrow = ((int64_t)b * Hq + h) * T + i;
     const float l = lacc[lrow];
     const float inv = 1.f / l;
@@ -682,8 +710,12 @@ cudaError_t launch_fwd_d(const Problem& pr, const void* q, const void* k, const 
     trace_end(kTraceFwdMain, st);
 
     const int64_t fth = pr.rows_q_active() * (D / 8);
-    fwd_finalize_kernel<D><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(
-        oacc, lacc, shift, pr.B, pr.T, pr.Hq, pr.q0, (__nv_bfloat16*)o, lse, nflag, flags);
+    if (fth < ((int64_t)1 << 31))
+        fwd_finalize_kernel<D, true><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(
+            oacc, lacc, shift, pr.B, pr.T, pr.Hq, pr.q0, (__nv_bfloat16*)o, lse, nflag, flags);
+    else
+        fwd_finalize_kernel<D, false><<<(unsigned)((fth + 255) / 256), 256, 0, st>>>(
+            oacc, lacc, shift, pr.B, pr.T, pr.Hq, pr.q0, (__nv_bfloat16*)o, lse, nflag, flags);
     count_launches(1);
     fwd_fallback_kernel<D><<<148, 128, 0, st>>>(qb, kb, (const __nv_bfloat16*)v, idx, nsel, pr.B,
                                                 pr.T, pr.Hq, pr.Hkv, pr.topk, pr.scale, nflag, flags,
