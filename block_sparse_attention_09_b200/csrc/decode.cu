@@ -228,20 +228,25 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __nv_bfloat16* _
         return;
     }
     const int n = idx[(int64_t)bg * topk + s];
-    // stage K and V rows of block n (16-byte pieces) and the G query rows
+    // stage K and V rows of block n (16-byte pieces) as two copy groups, and
+    // the G query rows: the scores need only K, so V is still arriving while
+    // they are computed
     constexpr int kPieces = D / 8;
-    for (int x = t; x < 128 * kPieces; x += 128) {
-        const int row = x / kPieces, c = x % kPieces;
-        const int j = n * 128 + row;
-        const bool ok = j <= i;
-        const int64_t off = (((int64_t)b * T + (ok ? j : 0)) * Hkv + g) * D + c * 8;
-        cp_async_16(smem_u32(ks + row * SM::kStride + c * 8), k + off, ok ? 16u : 0u);
-        cp_async_16(smem_u32(vs + row * SM::kStride + c * 8), v + off, ok ? 16u : 0u);
+    for (int half = 0; half < 2; ++half) {
+        const __nv_bfloat16* src = half == 0 ? k : v;
+        __nv_bfloat16* dst = half == 0 ? ks : vs;
+        for (int x = t; x < 128 * kPieces; x += 128) {
+            const int row = x / kPieces, c = x % kPieces;
+            const int j = n * 128 + row;
+            const bool ok = j <= i;
+            const int64_t off = (((int64_t)b * T + (ok ? j : 0)) * Hkv + g) * D + c * 8;
+            cp_async_16(smem_u32(dst + row * SM::kStride + c * 8), src + off, ok ? 16u : 0u);
+        }
+        cp_async_commit();
     }
-    cp_async_commit();
     for (int x = t; x < G * D; x += 128)
         qs[x] = __bfloat162float(q[((int64_t)b * Hq + g * G) * D + x]) * c1;
-    cp_async_wait<0>();
+    cp_async_wait<1>();   // this thread's K pieces have landed
     __syncthreads();
     // scores: thread t = key t of the block; K 16 bytes and q 16 bytes at a time
     const int j = n * 128 + t;
@@ -289,6 +294,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __nv_bfloat16* _
         for (int o = 16; o > 0; o >>= 1) bs += __shfl_xor_sync(0xffffffffu, bs, o);
         if (lane == 0) rsum[h * 4 + warp] = bs;
     }
+    cp_async_wait<0>();   // and the V pieces
     __syncthreads();
     // PV: thread t = head-dim index; P four keys at a time
     if (t < D) {
