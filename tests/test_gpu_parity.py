@@ -168,6 +168,24 @@ def test_selection_float_inputs():
     assert mism <= ig.shape[0] // 100
 
 
+@pytest.mark.parametrize("topk", [48, 72])
+def test_selection_both_shared_memory_layouts(topk):
+    """The selection kernel splits shared memory between key stages and the
+    maxima ring by topk: three stages and a deep ring while the heap is small
+    (topk 48 here), two stages and a short ring above that (topk 72).  Both
+    must select exactly what the oracle selects, for every row, over enough
+    key blocks (100) that the ring wraps many times."""
+    from block_sparse_attention_09_b200 import msa
+    cfg = Config("sel", B=1, T=12800, Hq=8, Hkv=2, d=64, dp=32, topk=topk)
+    inp = make_inputs(cfg, seed=11, exact_proxy=True, parts=("qp", "kp"))
+    dev = to_dev(inp)
+    idx, nsel = msa.proxy_select(dev["qp"], dev["kp"], topk, check=True)
+    m = O.Dims(B=cfg.B, T=cfg.T, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, dp=cfg.dp, topk=topk)
+    io, no, _ = O.select(m, inp["qp"].float().numpy(), inp["kp"].float().numpy())
+    assert np.array_equal(nsel.cpu().numpy(), no)
+    assert np.array_equal(idx.cpu().numpy(), io)
+
+
 def test_equal_scores_pick_lowest_blocks():
     cfg = Config("ties", B=1, T=1536, Hq=4, Hkv=1, d=64, dp=32, topk=4)
     inp = make_inputs(cfg, seed=2, exact_proxy=True)
