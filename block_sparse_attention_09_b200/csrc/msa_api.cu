@@ -172,6 +172,19 @@ int check_ws(const Problem& p, int which, void* ws, size_t ws_bytes, WsLayout* L
 
 bool empty(const Problem& p) { return p.B == 0 || p.T == 0 || p.q0 >= p.T; }
 
+// A shard with no query row (q_begin == T, with B and T > 0) enqueues no
+// kernel, but it still clears the workspace's status words, so that
+// msa_check_status and msa_fallback_rows describe this call and not an
+// earlier one.
+bool no_rows(const Problem& p) { return p.B > 0 && p.T > 0 && p.q0 >= p.T; }
+int clear_status(void* ws, const WsLayout& L, void* stream)
+{
+    int rc;
+    if ((rc = check_device()) != MSA_OK) return rc;
+    if (cudaMemsetAsync((uint8_t*)ws + L.status, 0, 256, (cudaStream_t)stream) != cudaSuccess) return MSA_ERR_LAUNCH;
+    return MSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -192,6 +205,7 @@ int msa_proxy_select(const msa_dims* dims, const void* qp, const void* kp, int32
     if (rc != MSA_OK) return rc;
     WsLayout L;
     if ((rc = check_ws(p, MSA_SELECT, ws, ws_bytes, &L)) != MSA_OK) return rc;
+    if (no_rows(p)) return clear_status(ws, L, stream);
     if (empty(p)) return MSA_OK;
     if (!qp || !kp || !idx || !nsel) return MSA_ERR_NULL_PTR;
     if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(idx, 16) || !aligned(nsel, 16) ||
@@ -219,6 +233,7 @@ int msa_fwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v
     WsLayout L;
     const bool mass = (flags & MSA_BLOCK_MASS) != 0;
     if ((rc = check_ws(p, mass ? MSA_PROXY_BWD : MSA_FWD, ws, ws_bytes, &L)) != MSA_OK) return rc;
+    if (no_rows(p)) return clear_status(ws, L, stream);
     if (empty(p)) return MSA_OK;
     if (!q || !k || !v || !idx || !nsel || !o || !lse) return MSA_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(idx, 16) || !aligned(nsel, 16) ||
@@ -257,7 +272,7 @@ int msa_bwd_ex(const msa_dims* dims, const void* q, const void* k, const void* v
     if (p.B > 0 && p.T > 0 && p.q0 >= p.T) {
         // no query row computed: the partial dK, dV are zero
         if (!dk || !dv) return MSA_ERR_NULL_PTR;
-        if ((rc = check_device()) != MSA_OK) return rc;
+        if ((rc = clear_status(ws, L, stream)) != MSA_OK) return rc;
         const size_t bytes = (size_t)p.B * p.T * p.Hkv * p.d * ((flags & MSA_DKV_F32) ? 4 : 2);
         if (cudaMemsetAsync(dk, 0, bytes, (cudaStream_t)stream) != cudaSuccess ||
             cudaMemsetAsync(dv, 0, bytes, (cudaStream_t)stream) != cudaSuccess)
@@ -322,6 +337,14 @@ int msa_proxy_bwd(const msa_dims* dims, const void* qp, const void* kp, const in
     if (rc != MSA_OK) return rc;
     WsLayout L;
     if ((rc = check_ws(p, MSA_PROXY_BWD, ws, ws_bytes, &L)) != MSA_OK) return rc;
+    if (no_rows(p)) {   // no query row: dkp is zero everywhere
+        if (!dkp) return MSA_ERR_NULL_PTR;
+        if ((rc = clear_status(ws, L, stream)) != MSA_OK) return rc;
+        if (cudaMemsetAsync(dkp, 0, sizeof(float) * (size_t)p.B * p.T * p.Hp * p.dp, (cudaStream_t)stream) !=
+            cudaSuccess)
+            return MSA_ERR_LAUNCH;
+        return MSA_OK;
+    }
     if (empty(p)) return MSA_OK;
     if (!qp || !kp || !idx || !nsel || !dqp || !dkp || !loss) return MSA_ERR_NULL_PTR;
     if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(idx, 16) || !aligned(nsel, 16) || !aligned(dqp, 16) ||

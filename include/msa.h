@@ -74,8 +74,11 @@ typedef struct msa_dims {
  * of one sequence add up.  Rows before q_begin of q, qp, dout, o and lse are
  * not read.  A rank owning query rows [r0, r1) of a sequence passes T = r1,
  * q_begin = r0, its rows in place and the keys 0 .. r1-1 (the causal prefix
- * its queries can see).  q_begin = T computes no row (msa_bwd then writes
- * zero dk/dv).  Decode requires q_begin = 0.
+ * its queries can see).  q_begin = T computes no row: no kernel runs and no
+ * tensor is read; msa_bwd writes zero dk/dv, msa_proxy_bwd zero dkp, and
+ * every entry point still clears the workspace's status words (so it needs
+ * the device), which msa_check_status then reports as MSA_OK.  Decode
+ * requires q_begin = 0.
  */
 
 enum msa_status {

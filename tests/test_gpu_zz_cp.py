@@ -93,3 +93,26 @@ def test_rows_before_q_begin_untouched():
     assert dk.dtype == torch.float32
     assert close(msa.f32_to_bf16(dk)[:, q0:], dk_full[:, q0:]) and close(msa.f32_to_bf16(dv)[:, q0:],
                                                                           dv_full[:, q0:])
+
+
+def test_empty_shard_computes_nothing():
+    """q_begin = T: a shard with no query rows.  The forward's outputs and
+    the dQ rows are left untouched, and the fp32 dK/dV partials are exactly
+    zero (no query contributes)."""
+    from block_sparse_attention_09_b200 import msa
+    cfg = Config("empty", B=1, T=768, Hq=4, Hkv=1, d=64, dp=32, topk=3)
+    x = {k: v.cuda() for k, v in make_inputs(cfg, seed=23, exact_proxy=True).items()}
+    T = cfg.T
+    msa.proxy_select(x["qp"], x["kp"], cfg.topk, q_begin=T, check=True)   # launches no tile
+    idx, nsel = msa.proxy_select(x["qp"], x["kp"], cfg.topk, check=True)
+    o = torch.full_like(x["q"], 7.0)
+    lse = torch.full((cfg.B, cfg.Hq, T), 7.0, device="cuda")
+    msa.fwd(x["q"], x["k"], x["v"], idx, nsel, out=(o, lse), q_begin=T, check=True)
+    dq = torch.full_like(x["q"], 7.0)
+    dk = torch.full(x["k"].shape, 7.0, dtype=torch.float32, device="cuda")
+    dv = torch.full_like(dk, 7.0)
+    msa.bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, idx, nsel, out=(dq, dk, dv), q_begin=T, dkv_f32=True,
+            check=True)
+    torch.cuda.synchronize()
+    assert bool((o == 7.0).all()) and bool((lse == 7.0).all()) and bool((dq == 7.0).all())
+    assert bool((dk == 0).all()) and bool((dv == 0).all())
