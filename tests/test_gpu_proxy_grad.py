@@ -82,3 +82,39 @@ def test_proxy_grad_shape_of_the_gradient():
             sc = x["kp"][0, n * 128:j1, 0].astype(np.float64) @ x["qp"][0, i, 0].astype(np.float64)
             argmaxes.add(n * 128 + int(np.argmax(sc)))
     assert set(nz.tolist()) <= argmaxes
+
+
+def test_proxy_grad_of_a_shard():
+    """q_begin: every call of the step restricted to the query rows from a
+    block boundary on (a context-parallel shard).  dqp and the loss of those
+    rows, and dkp from their contributions alone, against the oracle over
+    the same rows; rows before q_begin of dqp and loss are left untouched."""
+    from block_sparse_attention_09_b200 import msa
+    cfg = CASES["ragged_b2_g4"]
+    q0 = 512
+    inp = make_inputs(cfg, seed=33, exact_proxy=True)
+    dev = to_dev(inp)
+    idx, nsel = msa.proxy_select(dev["qp"], dev["kp"], cfg.topk, q_begin=q0, check=True)
+    dims = msa.make_dims(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.d, cfg.dp, cfg.topk, q_begin=q0)
+    ws = msa.proxy_workspace(dims, dev["q"].device)
+    o, lse = msa.fwd(dev["q"], dev["k"], dev["v"], idx, nsel, ws=ws, check=True, block_mass=True, q_begin=q0)
+    msa.bwd(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, idx, nsel, ws=ws, reuse_index=True, check=True,
+            q_begin=q0)
+    dqp = torch.full(dev["qp"].shape, 7.0, dtype=torch.float32, device="cuda")
+    dkp = torch.empty(dev["kp"].shape, dtype=torch.float32, device="cuda")
+    loss = torch.full((cfg.B, cfg.Hkv, cfg.T), 7.0, dtype=torch.float32, device="cuda")
+    msa.proxy_bwd(dev["q"], dev["qp"], dev["kp"], idx, nsel, ws, check=True, out=(dqp, dkp, loss), q_begin=q0)
+    torch.cuda.synchronize()
+    assert bool((dqp[:, :q0] == 7.0).all()) and bool((loss[:, :, :q0] == 7.0).all())
+    x = oracle_inputs(inp)
+    m = odims(cfg)
+    idx_o, nsel_o, _ = O.select(m, x["qp"], x["kp"])
+    gi, gn = idx.cpu().numpy(), nsel.cpu().numpy()
+    assert np.array_equal(gi[:, :, q0:], idx_o[:, :, q0:]) and np.array_equal(gn[:, :, q0:], nsel_o[:, :, q0:])
+    _, lse_o = O.fwd(m, x["q"], x["k"], x["v"], idx_o, nsel_o)
+    rows = [(b, g, i) for b in range(cfg.B) for g in range(cfg.Hkv) for i in range(q0, cfg.T)]
+    loss_o, dqp_o, dkp_o = PG.loss_and_grad(m, x["qp"], x["kp"], x["q"], x["k"], lse_o, idx_o, nsel_o, rows=rows)
+    tot = float(f32(loss)[:, :, q0:].astype(np.float64).sum())
+    assert abs(tot - loss_o) <= 1e-3 * abs(loss_o) + 2e-2, (tot, loss_o)
+    compare("dqp (shard)", f32(dqp)[:, q0:], dqp_o[:, q0:], rel=0.0)
+    compare("dkp (shard)", f32(dkp), dkp_o, rel=0.0)
