@@ -186,6 +186,22 @@ def test_selection_both_shared_memory_layouts(topk):
     assert np.array_equal(idx.cpu().numpy(), io)
 
 
+@pytest.mark.parametrize("dp", [8, 24, 40, 56])
+def test_selection_proxy_dims_not_multiple_of_16(dp):
+    """dp may be any multiple of 8 up to 64: the last K-step of the proxy MMA
+    then covers columns past dp, which the tensor map zero-fills.  The
+    selection must still match the oracle bit for bit (ragged T, B = 2)."""
+    from block_sparse_attention_09_b200 import msa
+    cfg = Config("dp", B=2, T=2000, Hq=4, Hkv=2, d=64, dp=dp, topk=5)
+    inp = make_inputs(cfg, seed=12, exact_proxy=True, parts=("qp", "kp"))
+    dev = to_dev(inp)
+    idx, nsel = msa.proxy_select(dev["qp"], dev["kp"], cfg.topk, check=True)
+    m = O.Dims(B=cfg.B, T=cfg.T, Hq=cfg.Hq, Hkv=cfg.Hkv, d=cfg.d, dp=dp, topk=cfg.topk)
+    io, no, _ = O.select(m, inp["qp"].float().numpy(), inp["kp"].float().numpy())
+    assert np.array_equal(nsel.cpu().numpy(), no)
+    assert np.array_equal(idx.cpu().numpy(), io)
+
+
 def test_equal_scores_pick_lowest_blocks():
     cfg = Config("ties", B=1, T=1536, Hq=4, Hkv=1, d=64, dp=32, topk=4)
     inp = make_inputs(cfg, seed=2, exact_proxy=True)
