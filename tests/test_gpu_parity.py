@@ -1,7 +1,7 @@
 """Parity of the CUDA path (through the C ABI) with the CPU oracle on shapes
-the oracle finishes in seconds: several tiles, ragged tails, every G the
-library supports, topk = 1, topk >= number of blocks, a sequence shorter
-than one block, B > 1.
+the oracle finishes in seconds: several tiles, ragged tails (down to a last
+block of one row), every G the library supports (1, 2, 4, 8, 16), topk = 1,
+topk >= number of blocks, a sequence shorter than one block, B > 1.
 
 Proxy inputs sit on the 1/8 grid (exact_proxy) so that the proxy scores are
 exact in any summation order: the GPU and the oracle then see identical
@@ -27,6 +27,7 @@ CASES = {
     "topk1": Config("topk1", B=1, T=640, Hq=4, Hkv=1, d=64, dp=32, topk=1),
     "short": Config("short", B=1, T=100, Hq=4, Hkv=1, d=64, dp=32, topk=2),
     "k5_ragged": Config("k5_ragged", B=1, T=1300, Hq=4, Hkv=1, d=128, dp=64, topk=5),
+    "g2_one_row_tail": Config("g2_one_row_tail", B=3, T=129, Hq=4, Hkv=2, d=128, dp=64, topk=2),
 }
 
 
