@@ -613,7 +613,13 @@ def main():
                  (torch.empty_like(o), torch.empty_like(lse), torch.empty_like(dq), torch.empty_like(dk),
                   torch.empty_like(dv))]
         hs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-        in_ready = [torch.cuda.Event() for _ in range(2)]
+        # the inputs go over in the order the step reads them (proxy pair, then
+        # q/k/v, then dout), each group with its own event, so the selection
+        # starts while the rest is still on its way; O goes back after the
+        # forward, the gradients after the backward
+        groups = (("qp", "kp"), ("q", "k", "v"), ("dout",))
+        in_ready = [[torch.cuda.Event() for _ in groups] for _ in range(2)]
+        fwd_done = [torch.cuda.Event() for _ in range(2)]
         comp_done = [torch.cuda.Event() for _ in range(2)]
         out_done = [torch.cuda.Event() for _ in range(2)]
 
@@ -626,23 +632,28 @@ def main():
                 if kk >= 2:
                     hs.wait_event(comp_done[sb])          # set sb's inputs no longer read
                 with torch.cuda.stream(hs):
-                    for name, v in host.items():          # this step's inputs
-                        d_in[sb][name].copy_(v, non_blocking=True)
-                    in_ready[sb].record(hs)
-                stream.wait_event(in_ready[sb])
+                    for gi, names in enumerate(groups):   # this step's inputs
+                        for name in names:
+                            d_in[sb][name].copy_(host[name], non_blocking=True)
+                        in_ready[sb][gi].record(hs)
                 if kk >= 2:
                     stream.wait_event(out_done[sb])       # set sb's outputs copied out
                 oo, ll, qq, kk_, vv = d_out[sb]
                 inp = d_in[sb]
+                stream.wait_event(in_ready[sb][0])
                 ix, ns = msa.proxy_select(inp["qp"], inp["kp"], cfg.topk, ws=ws_sel, window=args.window,
                                           dilation=args.dilation)
+                stream.wait_event(in_ready[sb][1])
                 msa.fwd(inp["q"], inp["k"], inp["v"], ix, ns, ws=ws_fwd, out=(oo, ll))
+                fwd_done[sb].record(stream)
+                stream.wait_event(in_ready[sb][2])
                 msa.bwd(inp["q"], inp["k"], inp["v"], oo, inp["dout"], ll, ix, ns, ws=ws_bwd, out=(qq, kk_, vv),
                         reuse_index=True)
                 comp_done[sb].record(stream)
-                ds.wait_event(comp_done[sb])
                 with torch.cuda.stream(ds):               # this step's results
+                    ds.wait_event(fwd_done[sb])
                     out_host["o"].copy_(oo, non_blocking=True)
+                    ds.wait_event(comp_done[sb])
                     out_host["dq"].copy_(qq, non_blocking=True)
                     out_host["dk"].copy_(kk_, non_blocking=True)
                     out_host["dv"].copy_(vv, non_blocking=True)
@@ -664,7 +675,8 @@ def main():
         e_ms, _ = combine_ranks(dist, world, dev, e_ms, f_step)
         e2e = {"value": f_job / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "pipelining": "two buffer sets; H2D, compute and D2H of neighbouring steps overlap"}
+               "pipelining": "two buffer sets; H2D, compute and D2H of neighbouring steps overlap; inputs copied "
+                               "in the order the step reads them, O copied back after the forward"}
 
     if world > 1:
         dist.barrier()
