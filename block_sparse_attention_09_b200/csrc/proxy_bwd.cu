@@ -361,11 +361,15 @@ __global__ void __launch_bounds__(256) proxy_grad_keys_kernel(
         int lent = 0, lkey = -1;
         float lw = 0.f;
         if (lane < 2 * kE && le < e1) {
+            // the three loads are independent: the weight and key slots exist for
+            // every entry and are used only when the entry selected the block
+            const int64_t x = (ebase + le) * 2 + lsb;
             lent = tok2[ebase + le];
+            const float w = dz[x];
+            const int key = jsel[x];
             if ((lent >> lsb) & 1) {
-                const int64_t x = (ebase + le) * 2 + lsb;
-                lw = dz[x];
-                lkey = jsel[x] - 256 * pn;   // 0 .. 255
+                lw = w;
+                lkey = key - 256 * pn;   // 0 .. 255
             }
         }
         float2 q[kE];
