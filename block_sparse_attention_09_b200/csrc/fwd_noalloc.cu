@@ -68,3 +68,11 @@ extern "C" int msa_fwd_noalloc(const msa_dims* dims, const void* q, const void* 
     if (rc != MSA_OK) return rc;
     return msa_fwd(dims, q, k, v, idx, nsel, o, lse, ws, msa::kNoAllocScratchBytes, stream);
 }
+
+extern "C" int msa_fwd_noalloc_status(void* stream, uint32_t* code)
+{
+    void* ws = nullptr;
+    const int rc = msa::scratch_on_current_device(&ws);
+    if (rc != MSA_OK) return rc == MSA_ERR_LAUNCH ? MSA_ERR_DEVICE : rc;
+    return msa_check_status(ws, stream, code);
+}

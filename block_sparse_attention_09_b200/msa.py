@@ -360,3 +360,13 @@ def fwd_noalloc(q, k, v, idx, nsel, scale=0.0, stream=None, out=None):
     _check(fn(ctypes.byref(dims), _p(q), _p(k), _p(v), _p(idx), _p(nsel), _p(o), _p(lse), _stream(stream)),
            "msa_fwd_noalloc")
     return o, lse
+
+
+def fwd_noalloc_status(stream=None) -> int:
+    """msa_fwd_noalloc_status: synchronise and read the status the last
+    fwd_noalloc on the current device left in the library's scratch."""
+    fn = LIB.msa_fwd_noalloc_status
+    fn.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
+    fn.restype = ctypes.c_int
+    code = ctypes.c_uint32(0)
+    return int(fn(_stream(stream), ctypes.byref(code)))

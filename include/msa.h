@@ -171,11 +171,22 @@ MSA_API int msa_bwd(const msa_dims* dims, const void* q, const void* k, const vo
  *  - All calls on a device share the array and it keeps the last call's
  *    contents (whatever must start at zero is cleared by every call).  Calls
  *    whose work overlaps on the GPU race on it: serialise them.
- *  - Device-side status (timeouts, malformed idx) stays in the shared array
- *    and is not reported; validate idx with msa_fwd when in doubt.
+ *  - Device-side status (timeouts, malformed idx) stays in the shared array;
+ *    msa_fwd_noalloc_status reads it.
  */
 MSA_API int msa_fwd_noalloc(const msa_dims* dims, const void* q, const void* k, const void* v,
                             const int32_t* idx, const int32_t* nsel, void* o, float* lse, void* stream);
+
+/*
+ * msa_check_status for msa_fwd_noalloc: synchronises `stream` and reads the
+ * status words that the last msa_fwd_noalloc on the current device left in
+ * the library's scratch array (every call clears them first).  Returns
+ * MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_INDEX (with *code as msa_check_status
+ * sets it; code may be NULL), MSA_ERR_LAUNCH if the stream or the copy
+ * failed, MSA_ERR_DEVICE if the scratch array cannot be found on the current
+ * device.  Before any msa_fwd_noalloc on the device it reports MSA_OK.
+ */
+MSA_API int msa_fwd_noalloc_status(void* stream, uint32_t* code);
 
 /*
  * Decode: attention of one new query token per sequence against caches, with

@@ -184,6 +184,17 @@ def test_q_begin_at_t_only_clears_the_status(lib):
                            ws, nb, None) == -2
 
 
+def test_noalloc_status_needs_a_device(lib):
+    """The no-alloc status read looks up the library's scratch array on the
+    current device; without a device it reports MSA_ERR_DEVICE."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    code = ctypes.c_uint32(7)
+    assert lib.LIB.msa_fwd_noalloc_status(None, ctypes.byref(code)) == -7
+    assert lib.LIB.msa_fwd_noalloc_status(None, None) == -7
+
+
 def test_f32_to_bf16_argument_checks(lib):
     P = 4096
     assert lib.LIB.msa_f32_to_bf16(P, P, 12, None) == -1      # not a multiple of 8

@@ -43,3 +43,21 @@ def test_fwd_noalloc_rejects_problems_beyond_its_scratch():
     assert msa.workspace_size(big, msa.MSA_FWD) > (64 << 20)
     P = ctypes.c_void_p(4096)
     assert fn(ctypes.byref(big), P, P, P, P, P, P, P, None) == -4
+
+
+def test_fwd_noalloc_status_reports_malformed_indices():
+    from block_sparse_attention_09_b200 import msa
+    cfg = Config("noalloc_bad", B=1, T=512, Hq=4, Hkv=1, d=64, dp=32, topk=2)
+    dev = {k: v.cuda() for k, v in make_inputs(cfg, seed=6).items()}
+    idx, nsel = msa.proxy_select(dev["qp"], dev["kp"], cfg.topk, check=True)
+    msa.fwd_noalloc(dev["q"], dev["k"], dev["v"], idx, nsel)
+    assert msa.fwd_noalloc_status() == 0
+    bad = idx.clone()
+    bad[0, 0, 300, 0] = 3        # a block after the query's own (300 // 128 = 2)
+    bad[0, 0, 10, 0] = -5
+    msa.fwd_noalloc(dev["q"], dev["k"], dev["v"], bad, nsel)   # the launch itself succeeds
+    assert msa.fwd_noalloc_status() == -9
+    # the next call clears the words it reports
+    o, _ = msa.fwd_noalloc(dev["q"], dev["k"], dev["v"], idx, nsel)
+    assert msa.fwd_noalloc_status() == 0
+    assert torch.isfinite(o.float()).all()
