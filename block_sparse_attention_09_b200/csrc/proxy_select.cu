@@ -8,10 +8,11 @@
 // One CTA owns one (batch, group, 128-query tile qb).  The proxy query tile
 // stays in shared memory; proxy key tiles n = 0 .. qb-1 stream in through a
 // TMA ring two key blocks at a time; one thread issues tcgen05 MMAs (M=128
-// queries, N=256 keys, K=dp: at N=128 an accumulation chain of dependent
-// MMAs runs at half rate) into two TMEM accumulators; eight pooling warps (one TMEM lane = one
-// query row each; two warps per lane quarter, one per key block of the
-// 256-key MMA) reduce each 128-column block to its max, free the
+// queries, N=256 keys, K=dp; one N=128 chain per block measured slower: twice
+// the MMAs and hand-offs for the same work) into two TMEM accumulators; eight
+// pooling warps (one TMEM lane = one query row each; two warps per lane
+// quarter, one per key block of the 256-key MMA) reduce each 128-column
+// block to its max, free the
 // accumulator and pass the maxima through a shared-memory ring to four
 // selection warps, which own the rows' selection state.  Pooling and
 // selection thus overlap, and the accumulator is handed back to the MMA as
